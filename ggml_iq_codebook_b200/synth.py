@@ -1,0 +1,149 @@
+"""Seeded synthetic inputs for the IQ encoder path.
+
+This module only draws random numbers: codebook grids, bf16 weights, per-column importance and
+block Hessians. It holds none of the encoder's arithmetic, so both the CUDA path and the CPU oracle
+take their inputs from here without sharing any of the method.
+
+Recipes (all seeded, all reproducible):
+
+* IQ1_S grid: 2048 distinct 8-vectors over {-1, 0, 1}, coordinates i.i.d. uniform, duplicates
+  rejected in draw order. The real GGML tables are third-party data and are not used.
+* IQ2_XS grid: 512 distinct 8-vectors over {1, 3, 5, 7}, drawn the same way.
+* Weights: i.i.d. normal in fp32, rounded to bf16 (round to nearest even). Outlier columns are
+  scaled by 8 after the rounding, which is exact in bf16.
+* Importance: per input column, log-normal(0, 1) in fp64, stored as fp32; the square-root
+  variant is the square root of a log-normal Hessian diagonal.
+* Block Hessian: H = U^-1 U^-T for an upper-triangular U with diagonal uniform in [0.5, 2] and
+  off-diagonal N(0, 0.02^2), computed in fp64, symmetrised, stored as fp32.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+GRID_SEED = 0x16C0DE
+BLOCK = 256
+
+IQ1S_GRID_ENTRIES = 2048
+IQ2XS_GRID_ENTRIES = 512
+
+
+def _distinct_rows(values: np.ndarray, n: int, seed: int) -> np.ndarray:
+    """Draw n distinct 8-vectors whose coordinates are uniform over `values`."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    seen: set[bytes] = set()
+    rows: list[np.ndarray] = []
+    while len(rows) < n:
+        batch = values[rng.integers(0, len(values), size=(4 * n, 8))]
+        for r in batch:
+            key = r.tobytes()
+            if key in seen:
+                continue
+            seen.add(key)
+            rows.append(r)
+            if len(rows) == n:
+                break
+    return np.ascontiguousarray(np.stack(rows).astype(np.int8))
+
+
+def iq1s_grid(seed: int = GRID_SEED) -> np.ndarray:
+    """[2048, 8] int8, entries in {-1, 0, 1}, all rows distinct."""
+    return _distinct_rows(np.array([-1, 0, 1], dtype=np.int8), IQ1S_GRID_ENTRIES, seed)
+
+
+def iq2xs_grid(seed: int = GRID_SEED + 1) -> np.ndarray:
+    """[512, 8] int8, entries in {1, 3, 5, 7}, all rows distinct."""
+    return _distinct_rows(np.array([1, 3, 5, 7], dtype=np.int8), IQ2XS_GRID_ENTRIES, seed)
+
+
+def normal_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
+    """i.i.d. N(0, std^2) drawn in fp32 on `device`, rounded to bf16."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return (x * std).to(torch.bfloat16)
+
+
+def outlier_columns(cols: int, frac: float, seed: int) -> torch.Tensor:
+    """A seeded choice of round(frac * cols) column indices."""
+    g = torch.Generator().manual_seed(seed)
+    n = int(round(frac * cols))
+    return torch.randperm(cols, generator=g)[:n].sort().values
+
+
+def with_outlier_columns(w: torch.Tensor, cols_idx: torch.Tensor, factor: float = 8.0) -> torch.Tensor:
+    """Scale the chosen columns by a power of two (exact in bf16)."""
+    w = w.clone()
+    w[..., cols_idx.to(w.device)] *= factor
+    return w
+
+
+def lognormal(shape, seed: int, device="cpu") -> torch.Tensor:
+    """log-normal(0, 1) values drawn in fp64, stored as fp32."""
+    g = torch.Generator().manual_seed(seed)
+    z = torch.randn(shape, generator=g, dtype=torch.float64)
+    return torch.exp(z).to(torch.float32).to(device)
+
+
+def sqrt_lognormal(shape, seed: int, device="cpu") -> torch.Tensor:
+    """Square root of a log-normal(0, 1) Hessian diagonal, fp64 then fp32."""
+    g = torch.Generator().manual_seed(seed)
+    z = torch.randn(shape, generator=g, dtype=torch.float64)
+    return torch.sqrt(torch.exp(z)).to(torch.float32).to(device)
+
+
+def block_hessian(seed: int, n: int = BLOCK, offdiag_std: float = 0.02) -> torch.Tensor:
+    """H = U^-1 U^-T (fp64, symmetrised) as fp32 [n, n]."""
+    g = torch.Generator().manual_seed(seed)
+    diag = 0.5 + 1.5 * torch.rand(n, generator=g, dtype=torch.float64)
+    off = offdiag_std * torch.randn((n, n), generator=g, dtype=torch.float64)
+    u = torch.triu(off, diagonal=1) + torch.diag(diag)
+    uinv = torch.linalg.solve_triangular(u, torch.eye(n, dtype=torch.float64), upper=True)
+    h = uinv @ uinv.T
+    h = 0.5 * (h + h.T)
+    return h.to(torch.float32).contiguous()
+
+
+# ---------------------------------------------------------------------------------------------
+# The five workloads. Each returns a dict of host (or `device`) tensors; names say what they are.
+# ---------------------------------------------------------------------------------------------
+
+def workload_iq1s_64x256(device="cpu"):
+    """IQ1_S, one 64x256 bf16 weight N(0, 0.02^2), uniform importance."""
+    return {
+        "fmt": "iq1_s",
+        "w": normal_bf16((64, 256), 0.02, 1001, device),
+        "importance": None,
+    }
+
+
+def workload_iq1s_4096x4096_weighted(device="cpu", rows=4096, cols=4096):
+    """IQ1_S weighted: N(0, 0.02^2) with 1% of columns x8, importance = sqrt(log-normal)."""
+    w = normal_bf16((rows, cols), 0.02, 1002, device)
+    w = with_outlier_columns(w, outlier_columns(cols, 0.01, 2002))
+    return {"fmt": "iq1_s", "w": w, "importance": sqrt_lognormal((cols,), 3002, device)}
+
+
+def workload_iq2xs_8192x4096(device="cpu", rows=8192, cols=4096):
+    """IQ2_XS: N(0, 0.015^2), per-column log-normal importance."""
+    return {
+        "fmt": "iq2_xs",
+        "w": normal_bf16((rows, cols), 0.015, 1003, device),
+        "importance": lognormal((cols,), 3003, device),
+    }
+
+
+def workload_iq1s_moe(device="cpu", experts=256, rows=1536, cols=4096):
+    """MoE batch: `experts` weights of rows x cols, N(0, 0.02^2), per-expert log-normal importance."""
+    return {
+        "fmt": "iq1_s",
+        "w": normal_bf16((experts, rows, cols), 0.02, 1004, device),
+        "importance": lognormal((experts, cols), 3004, device),
+    }
+
+
+def workload_choice_iq2xs(device="cpu", rows=4096, cols=4096):
+    """Local-Hessian choice search: N(0, 0.02^2) weight, one H per 256-column block."""
+    nblk = cols // BLOCK
+    hess = torch.stack([block_hessian(5000 + b) for b in range(nblk)]).to(device)
+    return {"fmt": "iq2_xs", "w": normal_bf16((rows, cols), 0.02, 1005, device), "hess": hess}

@@ -1,0 +1,183 @@
+"""CPU oracle for the GGML IQ encoder path -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ2_XS encoder, decoder and
+local-Hessian choice search, with this thin ctypes wrapper. It is the yardstick the CUDA library is
+checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import it; the library never does, and the two share no code.
+
+Functions whose parity rests on invariants only (no value fixed by the pages or by a closed form)
+are marked "parity unpinned" in their docstrings.
+"""
+
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "iq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+FMT = {"iq1_s": 1, "iq2_xs": 2}
+BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74}
+CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16}
+NUM_CHOICES = 16
+
+FLAG_NONFINITE = 1
+FLAG_IMPORTANCE = 2
+FLAG_RANGE = 4
+FLAG_CHOICE = 8
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile iq_oracle.c with gcc (-ffp-contract=off keeps a*b+c as two roundings)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-std=c11", "-O2", "-Wall", "-ffp-contract=off", "-fno-fast-math",
+               "-fopenmp", "-shared", "-fPIC", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load(path: str | None = None):
+    global _lib
+    if _lib is None or path is not None:
+        lib = ctypes.CDLL(path or build())
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.orc_encode.restype = ctypes.c_uint32
+        lib.orc_encode.argtypes = [ctypes.c_int, P, ctypes.c_float, P, i64, i64, P, P, ctypes.c_int, P]
+        lib.orc_decode.restype = None
+        lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
+        lib.orc_choice_search.restype = None
+        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, P, P, P, P]
+        lib.orc_sqrt_diag.restype = None
+        lib.orc_sqrt_diag.argtypes = [P, i64, P]
+        lib.orc_f32_to_f16.restype = ctypes.c_uint16
+        lib.orc_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.orc_f16_to_f32.restype = ctypes.c_float
+        lib.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.orc_f32_to_bf16_array.restype = None
+        lib.orc_f32_to_bf16_array.argtypes = [P, i64, P]
+        lib.orc_set_threads.argtypes = [ctypes.c_int]
+        lib.orc_get_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+@contextlib.contextmanager
+def library(path: str):
+    """Temporarily run every oracle call through another build of iq_oracle.c (used by the
+    mutation test, which plants mistakes in a copy of the source and expects the pins to fail)."""
+    global _lib
+    saved = _lib
+    _load(path)
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bf16_bits(w) -> np.ndarray:
+    """Accept a torch bf16 tensor or a uint16 array of bf16 bit patterns."""
+    if hasattr(w, "view") and hasattr(w, "dtype") and str(w.dtype) == "torch.bfloat16":
+        import torch
+        return np.ascontiguousarray(w.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    return np.ascontiguousarray(np.asarray(w, dtype=np.uint16))
+
+
+def set_threads(n: int) -> None:
+    _load().orc_set_threads(int(n))
+
+
+def threads() -> int:
+    return int(_load().orc_get_threads())
+
+
+def f32_to_f16_bits(v: float) -> int:
+    return int(_load().orc_f32_to_f16(float(v)))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(_load().orc_f16_to_f32(int(h)))
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty(a.shape, dtype=np.uint16)
+    _load().orc_f32_to_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choices=None,
+           every_choice: bool = False):
+    """Encode a [rows, cols] bf16 weight. Returns (payload uint8, flags).
+
+    payload: [rows, cols/256, B], or [16, rows, cols/256, B] with every_choice.
+    """
+    lib = _load()
+    wb = _bf16_bits(w)
+    rows, cols = wb.shape
+    if cols % 256:
+        raise ValueError("cols must be a multiple of 256")
+    nblk = cols // 256
+    B = BLOCK_BYTES[fmt]
+    grid = np.ascontiguousarray(grid, dtype=np.int8)
+    imp = None if importance is None else np.ascontiguousarray(np.asarray(importance, dtype=np.float32))
+    ch = None if choices is None else np.ascontiguousarray(np.asarray(choices, dtype=np.uint8))
+    shape = (NUM_CHOICES, rows, nblk, B) if every_choice else (rows, nblk, B)
+    out = np.zeros(shape, dtype=np.uint8)
+    flags = lib.orc_encode(FMT[fmt], _ptr(grid), float(anchor), _ptr(wb), rows, cols, _ptr(imp),
+                           _ptr(ch), int(bool(every_choice)), _ptr(out))
+    return out, int(flags)
+
+
+def decode(fmt: str, grid: np.ndarray, payload: np.ndarray) -> np.ndarray:
+    """Decode payload [..., B] to fp32 [..., 256] (exact)."""
+    B = BLOCK_BYTES[fmt]
+    p = np.ascontiguousarray(payload, dtype=np.uint8)
+    nblocks = p.size // B
+    out = np.empty(p.shape[:-1] + (256,), dtype=np.float32)
+    _load().orc_decode(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(p), nblocks, _ptr(out))
+    return out
+
+
+def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False):
+    """Local-Hessian choice search over every 256-column block of w.
+
+    hess: [nblk, 256, 256] fp32; cand: [16, rows, nblk, B] every-choice payloads.
+    Returns (picks [rows, nblk, G], payload [rows, nblk, B]) and, with trace, the picks after
+    step 2 and after each sweep [rows, nblk, 3, G].
+    Parity of the sweeps is pinned by the fp64 direct-objective replay in the tests.
+    """
+    wb = _bf16_bits(w)
+    rows, cols = wb.shape
+    nblk = cols // 256
+    G, B = CHOICE_GROUPS[fmt], BLOCK_BYTES[fmt]
+    hess = np.ascontiguousarray(hess, dtype=np.float32).reshape(nblk, 256, 256)
+    cand = np.ascontiguousarray(cand, dtype=np.uint8).reshape(NUM_CHOICES, rows, nblk, B)
+    picks = np.zeros((rows, nblk, G), dtype=np.uint8)
+    payload = np.zeros((rows, nblk, B), dtype=np.uint8)
+    tr = np.zeros((rows, nblk, 3, G), dtype=np.uint8) if trace else None
+    _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
+                              rows, nblk, cols, _ptr(hess), _ptr(cand), _ptr(picks), _ptr(payload),
+                              _ptr(tr))
+    return (picks, payload, tr) if trace else (picks, payload)
+
+
+def sqrt_diag(hess: np.ndarray) -> np.ndarray:
+    """sqrt of the diagonal of each [256, 256] block: the candidates' search importance."""
+    h = np.ascontiguousarray(hess, dtype=np.float32).reshape(-1, 256, 256)
+    out = np.empty((h.shape[0] * 256,), dtype=np.float32)
+    _load().orc_sqrt_diag(_ptr(h), h.shape[0], _ptr(out))
+    return out
