@@ -1,0 +1,239 @@
+"""Python binding of libiq_b200 (the B200 GGML IQ encoder library).
+
+Thin ctypes marshalling over the C ABI in include/iq.h: torch tensors supply device memory and
+the current CUDA stream, every computation runs in the library's kernels. There is no CPU path:
+if the shared library is missing or the device is not an sm_100 part, calls raise.
+
+Functions keep the C names: iq_encode, iq_decode, iq_choice_search, iq_sqrt_diag.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libiq_b200.so")
+
+IQ_FMT = {"iq1_s": 1, "iq2_xs": 2}
+BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74}
+CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16}
+GRID_ENTRIES = {"iq1_s": 2048, "iq2_xs": 512}
+NUM_CHOICES = 16
+# d = fp16(fp32(amax / qmax) * anchor): IQ1_S's 0.61 is the pages' constant; IQ2_XS's was fixed
+# once by a seeded sweep on non-evaluation data (the pages name a clamp but give no numbers).
+DEFAULT_ANCHOR = {"iq1_s": 0.61, "iq2_xs": 0.9}
+
+IQ_OUT_F32, IQ_OUT_BF16 = 0, 1
+FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
+
+SYMBOLS = ("iq_block_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
+           "iq_choice_search", "iq_sqrt_diag", "iq_status_string", "iq_build_info")
+
+
+class IQError(RuntimeError):
+    """A non-OK status from the library, or a device-side finding in the flags word."""
+
+
+class IQDesc(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("grid_entries", ctypes.c_int32),
+                ("grid", ctypes.c_void_p), ("anchor", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libiq_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise IQError(f"{path} is missing: build it with ggml_iq_codebook_b200.build.build()")
+    lib = ctypes.CDLL(path)
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    lib.iq_block_bytes.restype = ctypes.c_size_t
+    lib.iq_block_bytes.argtypes = [i32]
+    lib.iq_choice_groups.restype = i32
+    lib.iq_choice_groups.argtypes = [i32]
+    lib.iq_num_choices.restype = i32
+    lib.iq_num_choices.argtypes = [i32]
+    lib.iq_encode.restype = ctypes.c_int
+    lib.iq_encode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, i64, i64, P, i64, P, i32, P, P, P]
+    lib.iq_decode.restype = ctypes.c_int
+    lib.iq_decode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i32, P, P]
+    lib.iq_choice_search.restype = ctypes.c_int
+    lib.iq_choice_search.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, P, i64, i64, P, P, i64, P, P]
+    lib.iq_sqrt_diag.restype = ctypes.c_int
+    lib.iq_sqrt_diag.argtypes = [P, i64, P, P]
+    lib.iq_status_string.restype = ctypes.c_char_p
+    lib.iq_status_string.argtypes = [ctypes.c_int]
+    lib.iq_build_info.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise IQError(f"libiq_b200: {load_library().iq_status_string(status).decode()} (status {status})")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise IQError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise IQError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def make_desc(fmt: str, grid: torch.Tensor, anchor: float | None = None) -> IQDesc:
+    """Descriptor for a device grid ([2048, 8] or [512, 8] int8)."""
+    _need(grid, torch.int8, "grid")
+    if tuple(grid.shape) != (GRID_ENTRIES[fmt], 8) or not grid.is_contiguous():
+        raise IQError(f"grid must be a contiguous [{GRID_ENTRIES[fmt]}, 8] int8 tensor")
+    d = IQDesc(IQ_FMT[fmt], GRID_ENTRIES[fmt], grid.data_ptr(),
+               DEFAULT_ANCHOR[fmt] if anchor is None else float(anchor))
+    d._grid_ref = grid  # keep the device grid alive with the descriptor
+    return d
+
+
+def _fmt_of(desc: IQDesc) -> str:
+    return "iq1_s" if desc.fmt == 1 else "iq2_xs"
+
+
+def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = None,
+              choices: torch.Tensor | None = None, every_choice: bool = False,
+              out: torch.Tensor | None = None, flags: torch.Tensor | None = None, stream=None,
+              raise_on_flags: bool = True) -> torch.Tensor:
+    """Encode bf16 weights [rows, cols] or [batch, rows, cols] (last dim contiguous).
+
+    importance: fp32 [cols] or [batch, cols]; choices: uint8 [..., rows, cols/256, G].
+    Returns the payload uint8 [(16,) (batch,) rows, cols/256, B]. With raise_on_flags (default)
+    the call synchronises and raises on a device-side finding; pass a flags tensor and
+    raise_on_flags=False to stay asynchronous.
+    """
+    lib = load_library()
+    fmt = _fmt_of(desc)
+    _need(w, torch.bfloat16, "w")
+    batched = w.dim() == 3
+    if w.dim() not in (2, 3) or w.stride(-1) != 1:
+        raise IQError("w must be [rows, cols] or [batch, rows, cols] with a contiguous last dim")
+    batch = w.shape[0] if batched else 1
+    rows, cols = w.shape[-2], w.shape[-1]
+    ldw = w.stride(-2)
+    wbs = w.stride(0) if batched else 0
+    imp_ptr, imp_bs = None, 0
+    if importance is not None:
+        _need(importance, torch.float32, "importance")
+        if importance.stride(-1) != 1 or importance.shape[-1] != cols:
+            raise IQError("importance must be [cols] or [batch, cols] with a contiguous last dim")
+        imp_ptr = importance.data_ptr()
+        imp_bs = importance.stride(0) if importance.dim() == 2 else 0
+    ch_ptr = None
+    if choices is not None:
+        _need(choices, torch.uint8, "choices")
+        want = (batch, rows, cols // 256, CHOICE_GROUPS[fmt])
+        if choices.numel() != batch * rows * (cols // 256) * CHOICE_GROUPS[fmt] or not choices.is_contiguous():
+            raise IQError(f"choices must be a contiguous uint8 tensor of {want} elements")
+        ch_ptr = choices.data_ptr()
+    shape = ((NUM_CHOICES,) if every_choice else ()) + ((batch,) if batched else ()) + \
+        (rows, cols // 256, BLOCK_BYTES[fmt])
+    if out is None:
+        out = torch.empty(shape, dtype=torch.uint8, device=w.device)
+    elif tuple(out.shape) != shape or out.dtype != torch.uint8 or not out.is_contiguous():
+        raise IQError(f"out must be a contiguous uint8 tensor of shape {shape}")
+    if flags is None:
+        flags = torch.empty(1, dtype=torch.int32, device=w.device)
+    _check(lib.iq_encode(ctypes.byref(desc), w.data_ptr(), batch, rows, cols, ldw, wbs, imp_ptr, imp_bs,
+                         ch_ptr, int(bool(every_choice)), out.data_ptr(), flags.data_ptr(), _stream(stream)))
+    if raise_on_flags:
+        raise_for_flags(flags)
+    return out
+
+
+def raise_for_flags(flags: torch.Tensor) -> None:
+    """Synchronise on the flags word and raise if the kernels reported a finding."""
+    f = int(flags.item())
+    if f:
+        names = [n for n, b in (("non-finite weight", FLAG_NONFINITE), ("bad importance", FLAG_IMPORTANCE),
+                                ("d overflows fp16", FLAG_RANGE), ("choice out of range", FLAG_CHOICE),
+                                ("grid value outside the alphabet", FLAG_GRID)) if f & b]
+        err = IQError("device-side finding: " + ", ".join(names))
+        err.flags = f
+        raise err
+
+
+def iq_decode(desc: IQDesc, payload: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16,
+              out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode payload [..., B] to [..., 256] values (fp32 exact, or bf16)."""
+    lib = load_library()
+    fmt = _fmt_of(desc)
+    _need(payload, torch.uint8, "payload")
+    B = BLOCK_BYTES[fmt]
+    if payload.shape[-1] != B or not payload.is_contiguous():
+        raise IQError(f"payload must be contiguous with last dim {B}")
+    nblocks = payload.numel() // B
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise IQError("out_dtype must be float32 or bfloat16")
+    shape = tuple(payload.shape[:-1]) + (256,)
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=payload.device)
+    elif out.dtype != out_dtype or out.numel() != nblocks * 256 or not out.is_contiguous():
+        raise IQError("out has the wrong dtype or size")
+    _check(lib.iq_decode(ctypes.byref(desc), payload.data_ptr(), nblocks,
+                         IQ_OUT_BF16 if out_dtype == torch.bfloat16 else IQ_OUT_F32, out.data_ptr(),
+                         _stream(stream)))
+    return out
+
+
+def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor,
+                     picks: torch.Tensor | None = None, payload: torch.Tensor | None = None,
+                     flags: torch.Tensor | None = None, stream=None):
+    """Local-Hessian choice search over all 256-column blocks of w [rows, cols].
+
+    hess: fp32 [cols/256, 256, 256]; cand: uint8 [16, rows, cols/256, B] (every-choice payloads).
+    Returns (picks uint8 [rows, cols/256, G], payload uint8 [rows, cols/256, B]).
+    """
+    lib = load_library()
+    fmt = _fmt_of(desc)
+    _need(w, torch.bfloat16, "w")
+    _need(hess, torch.float32, "hess")
+    _need(cand, torch.uint8, "cand")
+    rows, cols = w.shape
+    nblk = cols // 256
+    B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
+    if w.stride(-1) != 1 or not hess.is_contiguous() or hess.numel() != nblk * 256 * 256:
+        raise IQError("w needs a contiguous last dim; hess must be contiguous [cols/256, 256, 256]")
+    if tuple(cand.shape) != (NUM_CHOICES, rows, nblk, B) or not cand.is_contiguous():
+        raise IQError(f"cand must be contiguous {(NUM_CHOICES, rows, nblk, B)}")
+    if picks is None:
+        picks = torch.empty((rows, nblk, G), dtype=torch.uint8, device=w.device)
+    if payload is None:
+        payload = torch.empty((rows, nblk, B), dtype=torch.uint8, device=w.device)
+    _check(lib.iq_choice_search(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(0), hess.data_ptr(),
+                                cand.data_ptr(), nblk, rows * nblk * B, picks.data_ptr(), payload.data_ptr(),
+                                nblk, None if flags is None else flags.data_ptr(), _stream(stream)))
+    return picks, payload
+
+
+def iq_sqrt_diag(hess: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """sqrt of the diagonal of each [256, 256] block: fp32 [nblk * 256]."""
+    lib = load_library()
+    _need(hess, torch.float32, "hess")
+    if not hess.is_contiguous() or hess.numel() % (256 * 256):
+        raise IQError("hess must be contiguous [nblk, 256, 256]")
+    nblk = hess.numel() // (256 * 256)
+    if out is None:
+        out = torch.empty(nblk * 256, dtype=torch.float32, device=hess.device)
+    _check(lib.iq_sqrt_diag(hess.data_ptr(), nblk, out.data_ptr(), _stream(stream)))
+    return out
+
+
+def build_info() -> str:
+    return load_library().iq_build_info().decode()

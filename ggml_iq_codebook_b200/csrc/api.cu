@@ -1,0 +1,184 @@
+// api.cu -- the C ABI (include/iq.h): argument validation on the host, then kernel launches.
+#include <atomic>
+#include <cmath>
+
+#include "iq.h"
+#include "iq_kernels.h"
+
+#define IQ_STR_(x) #x
+#define IQ_STR(x) IQ_STR_(x)
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];  // 0 unknown, -1 unsupported, >0 SM count
+
+// The current device must be an sm_100 part; returns its SM count (cached per device).
+iq_status device_sms(int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return IQ_ECUDA;
+    if (dev < 0 || dev >= kMaxDevices) return IQ_EUNSUPPORTED;
+    int v = g_sms[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        int major = 0, minor = 0, count = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return IQ_ECUDA;
+        v = (major == 10 && minor == 0) ? count : -1;
+        g_sms[dev].store(v, std::memory_order_relaxed);
+    }
+    if (v < 0) return IQ_EUNSUPPORTED;
+    *sms = v;
+    return IQ_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+iq_status check_desc(const iq_desc* d) {
+    if (d == nullptr || d->grid == nullptr) return IQ_EINVAL;
+    if (d->fmt == IQ_FMT_IQ1_S) {
+        if (d->grid_entries != 2048) return IQ_EINVAL;
+    } else if (d->fmt == IQ_FMT_IQ2_XS) {
+        if (d->grid_entries != 512) return IQ_EINVAL;
+    } else {
+        return IQ_EINVAL;
+    }
+    if (!aligned(d->grid, 16)) return IQ_EINVAL;
+    if (!std::isfinite(d->anchor) || !(d->anchor > 0.0f)) return IQ_EINVAL;
+    return IQ_OK;
+}
+
+iq_status launched(cudaError_t e) { return e == cudaSuccess ? IQ_OK : IQ_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t iq_block_bytes(int32_t fmt) {
+    return fmt == IQ_FMT_IQ1_S ? 50 : fmt == IQ_FMT_IQ2_XS ? 74 : 0;
+}
+
+int32_t iq_choice_groups(int32_t fmt) {
+    return fmt == IQ_FMT_IQ1_S ? 8 : fmt == IQ_FMT_IQ2_XS ? 16 : 0;
+}
+
+int32_t iq_num_choices(int32_t fmt) {
+    return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS) ? 16 : 0;
+}
+
+iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64_t rows, int64_t cols,
+                    int64_t ldw, int64_t w_batch_stride, const float* importance,
+                    int64_t imp_batch_stride, const uint8_t* choices, int32_t every_choice,
+                    uint8_t* payload, uint32_t* flags, cudaStream_t stream) {
+    iq_status st = check_desc(desc);
+    if (st != IQ_OK) return st;
+    if (w == nullptr || payload == nullptr) return IQ_EINVAL;
+    if (batch <= 0 || rows <= 0 || cols <= 0 || cols % 256 != 0) return IQ_ESHAPE;
+    if (ldw < cols || ldw % 8 != 0 || !aligned(w, 16)) return IQ_EINVAL;
+    if (batch > 1 && (w_batch_stride < (rows - 1) * ldw + cols || w_batch_stride % 8 != 0)) return IQ_EINVAL;
+    if (importance != nullptr) {
+        if (!aligned(importance, 16) || imp_batch_stride < 0 || imp_batch_stride % 4 != 0) return IQ_EINVAL;
+        if (batch > 1 && imp_batch_stride != 0 && imp_batch_stride < cols) return IQ_EINVAL;
+    }
+    if (every_choice != 0 && every_choice != 1) return IQ_EINVAL;
+    if (every_choice && choices != nullptr) return IQ_EINVAL;
+    if (!aligned(payload, 2)) return IQ_EINVAL;
+    int sms = 0;
+    if ((st = device_sms(&sms)) != IQ_OK) return st;
+    if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
+
+    iqk::EncodeParams p;
+    p.w = w;
+    p.rows = rows;
+    p.nblk = cols / 256;
+    p.ldw = ldw;
+    p.w_bstride = batch > 1 ? w_batch_stride : 0;
+    p.imp = importance;
+    p.imp_bstride = importance != nullptr ? imp_batch_stride : 0;
+    p.choices = choices;
+    p.payload = payload;
+    p.flags = flags;
+    p.grid = desc->grid;
+    p.anchor = desc->anchor;
+    p.nb = batch * rows * (cols / 256);
+    const int mode = every_choice ? iqk::kEvery : (choices != nullptr ? iqk::kFixed : iqk::kSearch);
+    return launched(desc->fmt == IQ_FMT_IQ1_S ? iqk::launch_iq1s_encode(p, mode, sms, stream)
+                                              : iqk::launch_iq2xs_encode(p, mode, sms, stream));
+}
+
+iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks, int32_t out_dtype,
+                    void* out, cudaStream_t stream) {
+    iq_status st = check_desc(desc);
+    if (st != IQ_OK) return st;
+    if (payload == nullptr || out == nullptr) return IQ_EINVAL;
+    if (nblocks <= 0) return IQ_ESHAPE;
+    if (out_dtype != IQ_OUT_F32 && out_dtype != IQ_OUT_BF16) return IQ_EINVAL;
+    if (!aligned(out, 16)) return IQ_EINVAL;
+    int sms = 0;
+    if ((st = device_sms(&sms)) != IQ_OK) return st;
+    iqk::DecodeParams p;
+    p.payload = payload;
+    p.nblocks = nblocks;
+    p.grid = desc->grid;
+    p.out = out;
+    return launched(iqk::launch_decode(desc->fmt, out_dtype == IQ_OUT_BF16, p, sms, stream));
+}
+
+iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows, int64_t nblk,
+                           int64_t ldw, const float* hess, const uint8_t* cand, int64_t cand_ld,
+                           int64_t cand_choice_stride, uint8_t* picks, uint8_t* payload,
+                           int64_t payload_ld, uint32_t* flags, cudaStream_t stream) {
+    iq_status st = check_desc(desc);
+    if (st != IQ_OK) return st;
+    if (w == nullptr || hess == nullptr || cand == nullptr || picks == nullptr || payload == nullptr)
+        return IQ_EINVAL;
+    if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;
+    if (ldw < nblk * 256 || ldw % 8 != 0 || !aligned(w, 16) || !aligned(hess, 16)) return IQ_EINVAL;
+    if (cand_ld < nblk || payload_ld < nblk || cand_choice_stride < 0) return IQ_EINVAL;
+    int sms = 0;
+    if ((st = device_sms(&sms)) != IQ_OK) return st;
+    if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
+    iqk::ChoiceParams p;
+    p.w = w;
+    p.rows = rows;
+    p.nblk = nblk;
+    p.ldw = ldw;
+    p.hess = hess;
+    p.cand = cand;
+    p.cand_ld = cand_ld;
+    p.cand_cstride = cand_choice_stride;
+    p.picks = picks;
+    p.payload = payload;
+    p.payload_ld = payload_ld;
+    p.flags = flags;
+    p.grid = desc->grid;
+    return launched(iqk::launch_choice_search(desc->fmt, p, sms, stream));
+}
+
+iq_status iq_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t stream) {
+    if (hess == nullptr || out == nullptr) return IQ_EINVAL;
+    if (nblk <= 0) return IQ_ESHAPE;
+    int sms = 0;
+    iq_status st = device_sms(&sms);
+    if (st != IQ_OK) return st;
+    return launched(iqk::launch_sqrt_diag(hess, nblk, out, stream));
+}
+
+const char* iq_status_string(iq_status s) {
+    switch (s) {
+        case IQ_OK: return "ok";
+        case IQ_EINVAL: return "invalid argument";
+        case IQ_ESHAPE: return "invalid shape (empty, or columns not a multiple of 256)";
+        case IQ_ECUDA: return "CUDA error";
+        case IQ_EUNSUPPORTED: return "device is not sm_100";
+        default: return "unknown status";
+    }
+}
+
+const char* iq_build_info(void) {
+    return "libiq_b200: nvcc " IQ_STR(__CUDACC_VER_MAJOR__) "." IQ_STR(__CUDACC_VER_MINOR__)
+           ", sm_100a, -fmad=false; encode: warp per block, lane per group, persistent CTAs";
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// iq_kernels.h -- internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime_api.h>
+#include <stdint.h>
+
+namespace iqk {
+
+enum EncodeMode { kSearch = 0, kFixed = 1, kEvery = 2 };
+
+struct EncodeParams {
+    const uint16_t* w;
+    int64_t rows, nblk, ldw, w_bstride;
+    const float* imp;  // nullptr: all ones
+    int64_t imp_bstride;
+    const uint8_t* choices;  // kFixed only
+    uint8_t* payload;
+    uint32_t* flags;
+    const int8_t* grid;
+    float anchor;
+    int64_t nb;  // batch * rows * nblk
+};
+
+struct DecodeParams {
+    const uint8_t* payload;
+    int64_t nblocks;
+    const int8_t* grid;
+    void* out;
+};
+
+struct ChoiceParams {
+    const uint16_t* w;
+    int64_t rows, nblk, ldw;
+    const float* hess;
+    const uint8_t* cand;
+    int64_t cand_ld, cand_cstride;
+    uint8_t* picks;
+    uint8_t* payload;
+    int64_t payload_ld;
+    uint32_t* flags;
+    const int8_t* grid;
+};
+
+// Each returns the cudaError_t of its launch (cudaSuccess when nothing had to run).
+cudaError_t launch_iq1s_encode(const EncodeParams& p, int mode, int num_sms, cudaStream_t s);
+cudaError_t launch_iq2xs_encode(const EncodeParams& p, int mode, int num_sms, cudaStream_t s);
+cudaError_t launch_decode(int fmt, bool bf16, const DecodeParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_choice_search(int fmt, const ChoiceParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t s);
+
+}  // namespace iqk

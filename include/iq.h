@@ -1,0 +1,165 @@
+/*
+ * iq.h -- C ABI of the B200 GGML IQ encoder library (libiq_b200.so).
+ *
+ * What the library computes (Model-Optimizer pull-request pages):
+ *   - IQ1_S and IQ2_XS weight encoding: every 256-weight super-block of a row is split into
+ *     8-weight groups; each group gets an exhaustive, importance-weighted codebook search that
+ *     minimises sum_j w_j (x_j - xhat_j)^2 over grid entry, sign/shift and local scale, and the
+ *     block is packed into its fixed byte layout. Sources: PR #2723 "Weight the IQ1 encoders by
+ *     the square root of GPTQ's Hessian diagonal" (objective, delta = +-1/8, unweighted d);
+ *     PR #2450 "[OMNIML-5899] Add IQ tests and release notes", review comments (IQ1_S 50-byte and
+ *     IQ2_XS 74-byte layouts, d = fp16((amax / 16.875) * 0.61), 16-way choice, lowest index wins
+ *     on equal error, even sign parity); the IQ2_S codec commit text on the PR #2525 page
+ *     (IQ2_XS fixes parity by flipping the weakest element).
+ *   - fixed per-group choices (PR #3157) and the one-pass every-choice encode (PR #3159);
+ *   - decoding of both layouts;
+ *   - the local-Hessian choice search (PR #3158, fused in PR #3218 "[4/4] Run the local-Hessian
+ *     choice search as one CUDA kernel").
+ *
+ * The exact floating-point op sequence of every score is a fixed convention (it is what makes
+ * payloads and picks bit-reproducible); it is documented next to each kernel.
+ *
+ * Memory: every pointer argument is DEVICE memory owned by the caller, except `desc`, which is a
+ * host struct. The library never allocates device memory. Calls are asynchronous on `stream`:
+ * they validate their arguments on the host, enqueue kernels and return. A non-IQ_OK status
+ * means nothing was enqueued (except IQ_ECUDA, reported after a failed launch).
+ *
+ * Device-side findings (non-finite weights, bad importance, out-of-range choices, d overflowing
+ * fp16, a grid value outside the format's alphabet) cannot be known on the host. The kernels OR
+ * IQ_FLAG_* bits into `*flags` (a caller-owned device uint32; the call first clears it, so after
+ * the stream reaches the end of the call it holds exactly this call's findings). Blocks with a
+ * finding are written as the all-zero payload. `flags` may be NULL to skip reporting.
+ *
+ * Requires an sm_100 (B200-class) device; other devices get IQ_EUNSUPPORTED.
+ */
+#ifndef IQ_B200_H
+#define IQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    IQ_OK = 0,
+    IQ_EINVAL = 1,        /* NULL pointer, unknown format, bad descriptor or stride          */
+    IQ_ESHAPE = 2,        /* empty tensor, or cols not a multiple of 256 ([512, 384] case)     */
+    IQ_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed                       */
+    IQ_EUNSUPPORTED = 4   /* the current device is not sm_100                                  */
+} iq_status;
+
+typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2 } iq_format;
+
+typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
+
+/* device-side findings, ORed into *flags */
+#define IQ_FLAG_NONFINITE 1u  /* a weight is NaN or +-inf                                 */
+#define IQ_FLAG_IMPORTANCE 2u /* an importance value is NaN, +-inf or negative            */
+#define IQ_FLAG_RANGE 4u      /* the block scale d rounds to fp16 infinity                 */
+#define IQ_FLAG_CHOICE 8u     /* a given choice is >= 16                                  */
+#define IQ_FLAG_GRID 16u      /* a grid value lies outside the format's alphabet           */
+
+/*
+ * Codebook/convention descriptor (host struct; the grid it points to lives on the device).
+ *   fmt           IQ_FMT_IQ1_S or IQ_FMT_IQ2_XS
+ *   grid_entries  2048 (IQ1_S) or 512 (IQ2_XS)
+ *   grid          device int8 [grid_entries][8]; IQ1_S values in {-1,0,1} (a ternary grid,
+ *                 PR #2723), IQ2_XS magnitudes in {1,3,5,7}. Row q, column j multiplies weight j
+ *                 of a group.
+ *   anchor        the scale predictor's anchor: d = fp16(fp32(amax / qmax) * anchor), with
+ *                 qmax = 16.875 (IQ1_S, = 15 * 1.125, the largest |s (q + delta)| in units of d)
+ *                 and 217 (IQ2_XS, = 31 * 7). IQ1_S uses 0.61 (PR #2450 review). The pages give
+ *                 no IQ2_XS constant; this library's default is 0.9.
+ */
+typedef struct {
+    int32_t fmt;
+    int32_t grid_entries;
+    const int8_t *grid;
+    float anchor;
+} iq_desc;
+
+/* Bytes per 256-weight block: 50 (IQ1_S), 74 (IQ2_XS); 0 for an unknown format. */
+size_t iq_block_bytes(int32_t fmt);
+
+/* Choice groups per block: 8 (IQ1_S, one per 32 weights: local scale + delta sign),
+ * 16 (IQ2_XS, one 4-bit local scale per 16 weights); 0 for an unknown format. */
+int32_t iq_choice_groups(int32_t fmt);
+
+/* Choices per group: 16 for both formats (IQ1_S: c = ls + 8 * [delta < 0]; IQ2_XS: c = ls). */
+int32_t iq_num_choices(int32_t fmt);
+
+/*
+ * Encode `batch` weights of [rows, cols] bf16 (bit patterns as uint16).
+ *   w[e * w_batch_stride + r * ldw + col]        (elements; ldw >= cols)
+ *   importance: NULL (all ones) or fp32 per input column,
+ *     importance[e * imp_batch_stride + col]     (imp_batch_stride 0 shares one vector)
+ *     values must be finite and >= 0 (PR #2723 review), else IQ_FLAG_IMPORTANCE.
+ *   choices: NULL, or uint8 [batch][rows][cols/256][G] forcing each choice group's choice
+ *     (PR #3157); entries and signs are still searched under it.
+ *   every_choice: 0, or 1 to write all 16 choices' payloads in one sweep (PR #3159):
+ *     payload c equals the encode with choices = full(c). Must be 0 when choices != NULL.
+ *   payload: uint8 [batch][rows][cols/256][B], or [16][batch][rows][cols/256][B] with every_choice.
+ * Per block ([#2450] layouts):
+ *   IQ1_S  bytes 0-1 fp16 d; 2..33 low 8 bits of the 32 group indices; 34..49 eight LE uint16 qh,
+ *          one per 32-weight sub-block: bits 0..11 the high 3 index bits of its 4 groups (shifts
+ *          0,3,6,9), bits 12..14 local scale ls, bit 15 set for delta = -1/8.
+ *   IQ2_XS bytes 0-1 fp16 d; 2..65 32 LE uint16 codes (9-bit index | 7-bit sign mask << 9, the
+ *          8th sign by even parity); 66..73 sixteen 4-bit local scales, sub-block 2i in the low
+ *          nibble of byte 66+i.
+ * Value of a weight: IQ1_S d (2 ls + 1)(q + delta); IQ2_XS d (2 ls + 1) g sign.
+ * amax == 0, or d rounding to fp16 zero, gives the all-zero payload ([#2450]).
+ */
+iq_status iq_encode(const iq_desc *desc, const uint16_t *w, int64_t batch, int64_t rows, int64_t cols,
+                    int64_t ldw, int64_t w_batch_stride, const float *importance,
+                    int64_t imp_batch_stride, const uint8_t *choices, int32_t every_choice,
+                    uint8_t *payload, uint32_t *flags, cudaStream_t stream);
+
+/*
+ * Decode nblocks contiguous payload blocks into [nblocks][256] values, fp32 (exact) or bf16
+ * (round to nearest even of the exact value). Output is independent of how blocks are chunked.
+ */
+iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks, int32_t out_dtype,
+                    void *out, cudaStream_t stream);
+
+/*
+ * Local-Hessian choice search (PR #3158 steps; one fused launch as in PR #3218) for the first
+ * nblk 256-column blocks of a [rows, ldw] bf16 weight.
+ *   hess: fp32 [nblk][256][256], the symmetric diagonal block of the input Hessian per block,
+ *     read as H[k][i] (row k, column i) for (H v)_i.
+ *   cand: the every-choice payloads of those blocks; candidate c of (row r, block b) starts at
+ *     cand + c * cand_choice_stride + (r * cand_ld + b) * B   (bytes; cand_ld in blocks).
+ *   picks: uint8 [rows][nblk][G], the chosen choice of every choice group.
+ *   payload: the final payload, block (r, b) at payload + (r * payload_ld + b) * B: each choice
+ *     group's fields copied from its picked candidate, d from candidate 0 (the encode under the
+ *     picks, PR #3157).
+ * Steps per (row, block): Delta(c) = x - decode(cand c); each group takes its best choice under
+ * its own H_gg; grad = H Delta; two sweeps over the groups in order, each taking the choice with
+ * the least gain 2 u^T grad_g + u^T H_gg u (u = Delta_g(c) - Delta_g(cur)) iff that gain < 0,
+ * then grad += H[:, g] u. Lowest choice on equal score or gain.
+ */
+iq_status iq_choice_search(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t nblk,
+                           int64_t ldw, const float *hess, const uint8_t *cand, int64_t cand_ld,
+                           int64_t cand_choice_stride, uint8_t *picks, uint8_t *payload,
+                           int64_t payload_ld, uint32_t *flags, cudaStream_t stream);
+
+/*
+ * out[b * 256 + i] = sqrtf(hess[b][i][i]) for b < nblk: the search importance the local-Hessian
+ * calibration uses for the every-choice candidates (square root of the Hessian diagonal, PR #3158).
+ */
+iq_status iq_sqrt_diag(const float *hess, int64_t nblk, float *out, cudaStream_t stream);
+
+/* A static, human-readable name for a status code. */
+const char *iq_status_string(iq_status s);
+
+/* Build information: compiler, target architecture, kernel configuration. */
+const char *iq_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IQ_B200_H */

@@ -1,0 +1,80 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no kernel launched)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import ggml_iq_codebook_b200 as iq
+from ggml_iq_codebook_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return iq.load_library()
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "iq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(iq_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert set(_declared_functions()) == set(iq.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_format_tables(lib):
+    assert lib.iq_block_bytes(1) == 50 and lib.iq_block_bytes(2) == 74 and lib.iq_block_bytes(3) == 0
+    assert lib.iq_choice_groups(1) == 8 and lib.iq_choice_groups(2) == 16
+    assert lib.iq_num_choices(1) == 16 and lib.iq_num_choices(2) == 16 and lib.iq_num_choices(0) == 0
+    assert b"sm_100a" in lib.iq_build_info()
+    assert lib.iq_status_string(2).startswith(b"invalid shape")
+
+
+def _desc(fmt=1, entries=2048, grid=0x1000, anchor=0.61):
+    return iq.IQDesc(fmt, entries, grid, anchor)
+
+
+def test_argument_errors_are_reported_before_any_launch(lib):
+    E = lib.iq_encode
+    d = _desc()
+    W = 0x10000  # a fake, 16-byte aligned address: validation must fail before it is touched
+    # bad descriptors
+    assert E(None, W, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=3)), W, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(anchor=float("nan"))), W, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(anchor=0.0)), W, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(grid=0x1001)), W, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    # shapes: the [512, 384] case, empty tensors
+    assert E(ctypes.byref(d), W, 1, 512, 384, 384, 0, None, 0, None, 0, W, None, None) == 2
+    assert E(ctypes.byref(d), W, 1, 0, 256, 256, 0, None, 0, None, 0, W, None, None) == 2
+    assert E(ctypes.byref(d), W, 0, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 2
+    # NULL buffers, strides, exclusive options
+    assert E(ctypes.byref(d), None, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 1, 4, 256, 128, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W + 2, 1, 4, 256, 256, 0, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 2, 4, 256, 256, 256, None, 0, None, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 1, 4, 256, 256, 0, None, 0, W, 1, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 1, 4, 256, 256, 0, None, 0, None, 2, W, None, None) == 1
+    # decode / choice search / sqrt_diag
+    assert lib.iq_decode(ctypes.byref(d), W, 0, 1, W, None) == 2
+    assert lib.iq_decode(ctypes.byref(d), W, 4, 7, W, None) == 1
+    assert lib.iq_decode(ctypes.byref(d), None, 4, 1, W, None) == 1
+    assert lib.iq_choice_search(ctypes.byref(d), W, 0, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 2
+    assert lib.iq_choice_search(ctypes.byref(d), W, 4, 2, 256, W, W, 2, 0, W, W, 2, None, None) == 1
+    assert lib.iq_sqrt_diag(None, 1, W, None) == 1
+    assert lib.iq_sqrt_diag(W, 0, W, None) == 2
