@@ -1,0 +1,511 @@
+#!/usr/bin/env python
+"""Benchmark of the IQ encoder hot path; rank 0 prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+A step is one pass of the hot path over one batch of synthetic input already resident in HBM.
+Default workload: IQ1_S importance-weighted encode of a 4096x4096 bf16 weight (N(0, 0.02^2), 1% of
+columns x8, importance = sqrt of a log-normal Hessian diagonal) followed by the decode of its
+payload. `value` is weights per second of the whole step (Mweights/s), timed with CUDA events on
+the launching stream around the library calls, the L2 cache flushed before every step.
+
+Multi-GPU (torchrun): every rank encodes its own copy of the workload (independent problems, no
+data-path collective): weak scaling, time = max over ranks.
+
+--impl reference times the CPU oracle on the host cores (a bounded sample of the same workload per
+step); it is the reference arm. It runs on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ggml_iq_codebook_b200 as iq  # noqa: E402
+from ggml_iq_codebook_b200 import synth  # noqa: E402
+
+METRIC = "IQ encode Mweights/s"
+UNIT = "Mweights/s"
+L2_FLUSH_BYTES = 256 << 20
+
+# FP32-pipe operations the method itself requires (the exhaustive search counts every candidate):
+#   IQ1_S, per (group, grid entry): 4 subset-sum adds + A, R, C (3) + A_delta, C_delta for both
+#     shifts (6 fma) = 13 term ops, then 16 choices x (1 fma score + 1 min) = 32 -> 45 ops;
+#     per 256-weight block: 32 groups x 2048 entries x 45 = 2,949,120 ops.
+#   IQ2_XS, per (group, entry): A and B chains (16) + 16 x (fma + min) = 48 ops;
+#     per block: 32 x 512 x 48 = 786,432 ops.
+#   Choice search (IQ2_XS, 16 groups of 16 columns, 16 choices), per row and block:
+#     own-block scores 16 x 16 x (256 + 16 + 15), gradient 256 x 256, two sweeps of
+#     16 groups x 16 choices x (256 + 5 x 16 - 1) gains; gradient updates after a switch are
+#     data dependent and not counted: 310,528 ops.
+OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432}
+CHOICE_OPS_PER_ROW_BLOCK = 310_528
+SMS, FP32_LANES = 148, 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def alu_peak_tops(mhz: float) -> float:
+    return SMS * FP32_LANES * mhz * 1e6 / 1e12
+
+
+def kernel_traffic(name: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(name)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
+        return None
+    return rec["bytes_per_launch"]
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_index: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = [v.strip() for v in vis.split(",")] if vis else None
+        self.index = ids[local_index] if ids and local_index < len(ids) else str(local_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        mhz, maxmhz, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxmhz = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": maxmhz, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------------------------ workloads
+
+class Workload:
+    """Inputs on the device plus one hot-path step; `units` weights per step."""
+
+    def __init__(self, name: str, dev, peaks):
+        self.name, self.dev, self.peaks = name, dev, peaks
+        g1 = torch.from_numpy(synth.iq1s_grid()).to(dev)
+        g2 = torch.from_numpy(synth.iq2xs_grid()).to(dev)
+        self.desc = {"iq1_s": iq.make_desc("iq1_s", g1), "iq2_xs": iq.make_desc("iq2_xs", g2)}
+        self.launches_per_step = 2
+        if name == "iq1s_4096x4096_weighted":
+            wl = synth.workload_iq1s_4096x4096_weighted()
+            self._encode_decode(wl, "IQ1_S importance-weighted encode + bf16 decode, 4096x4096 bf16 "
+                                    "N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))")
+        elif name == "iq2xs_8192x4096":
+            wl = synth.workload_iq2xs_8192x4096()
+            self._encode_decode(wl, "IQ2_XS importance-weighted encode + bf16 decode, 8192x4096 bf16 "
+                                    "N(0,0.015^2), importance lognormal(0,1)")
+        elif name == "iq1s_moe_256x1536x4096":
+            wl = synth.workload_iq1s_moe(device=dev)
+            self._encode_decode(wl, "IQ1_S weighted encode of 256 experts x 1536x4096 bf16 in one call "
+                                    "+ bf16 decode, importance lognormal(0,1) per expert")
+        elif name == "iq1s_64x256":
+            wl = synth.workload_iq1s_64x256()
+            self._encode_decode(wl, "IQ1_S encode + bf16 decode, one 64x256 bf16 weight, uniform importance")
+        elif name == "choice_iq2xs_4096x4096":
+            self._choice(synth.workload_choice_iq2xs())
+        elif name == "iq1s_decode_1m_blocks":
+            wl = synth.workload_iq1s_4096x4096_weighted()
+            self._encode_decode(wl, "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 weighted payload x16)")
+            self.kind = "decode"
+            self.payload = self.payload.reshape(-1, 50).repeat(16, 1)
+            self.decoded = torch.empty((self.payload.shape[0], 256), dtype=torch.bfloat16, device=self.dev)
+            self.units = self.payload.shape[0] * 256
+            self.nblocks = self.payload.shape[0]
+            self.launches_per_step = 1
+            self.dominant = "decode_kernel"
+            self.ops_per_launch = None
+        else:
+            raise SystemExit(f"unknown workload {name}")
+
+    def _encode_decode(self, wl, text):
+        self.fmt = wl["fmt"]
+        self.kind = "encode"
+        self.w_host = wl["w"]
+        self.imp_host = wl["importance"]
+        self.w = wl["w"].to(self.dev)
+        self.imp = None if wl["importance"] is None else wl["importance"].to(self.dev)
+        shape = tuple(self.w.shape[:-1]) + (self.w.shape[-1] // 256, iq.BLOCK_BYTES[self.fmt])
+        self.payload = torch.empty(shape, dtype=torch.uint8, device=self.dev)
+        self.decoded = torch.empty(tuple(self.w.shape[:-1]) + (self.w.shape[-1],), dtype=torch.bfloat16,
+                                   device=self.dev)
+        self.units = self.w.numel()
+        self.nblocks = self.units // 256
+        self.text = text
+        self.dominant = f"{self.fmt.replace('_', '')}_encode_kernel"
+        self.ops_per_launch = self.nblocks * OPS_PER_BLOCK[self.fmt]
+        # validate once (findings word + raise) before anything is timed
+        iq.iq_encode(self.desc[self.fmt], self.w, self.imp, out=self.payload)
+
+    def _choice(self, wl):
+        self.fmt, self.kind = "iq2_xs", "choice"
+        self.w_host, self.hess_host = wl["w"], wl["hess"]
+        self.w, self.hess = wl["w"].to(self.dev), wl["hess"].to(self.dev)
+        rows, cols = self.w.shape
+        nblk = cols // 256
+        self.imp = torch.empty(cols, dtype=torch.float32, device=self.dev)
+        self.cand = torch.empty((16, rows, nblk, 74), dtype=torch.uint8, device=self.dev)
+        self.picks = torch.empty((rows, nblk, 16), dtype=torch.uint8, device=self.dev)
+        self.payload = torch.empty((rows, nblk, 74), dtype=torch.uint8, device=self.dev)
+        self.units = self.w.numel()
+        self.nblocks = rows * nblk
+        self.launches_per_step = 3
+        self.text = ("local-Hessian choice search, IQ2_XS: sqrt(diag H) + one-pass every-choice encode + "
+                     "two-sweep search, 4096x4096 bf16 N(0,0.02^2), 16 blocks of H = U^-1 U^-T")
+        self.dominant = "choice_search_kernel"
+        self.ops_per_launch = rows * nblk * CHOICE_OPS_PER_ROW_BLOCK
+        iq.iq_sqrt_diag(self.hess, out=self.imp)
+        iq.iq_encode(self.desc["iq2_xs"], self.w, self.imp, every_choice=True, out=self.cand)
+
+    # one step; `ev` is a list of (start, end) event pairs to fill around the dominant kernel
+    def step(self, ev=None):
+        d = self.desc[self.fmt]
+        if self.kind == "decode":
+            if ev is not None:
+                ev[0].record()
+            iq.iq_decode(d, self.payload, torch.bfloat16, out=self.decoded)
+            if ev is not None:
+                ev[1].record()
+        elif self.kind == "encode":
+            if ev is not None:
+                ev[0].record()
+            iq.iq_encode(d, self.w, self.imp, out=self.payload, flags=False)
+            if ev is not None:
+                ev[1].record()
+            iq.iq_decode(d, self.payload, torch.bfloat16, out=self.decoded)
+        else:
+            iq.iq_sqrt_diag(self.hess, out=self.imp)
+            iq.iq_encode(d, self.w, self.imp, every_choice=True, out=self.cand, flags=False)
+            if ev is not None:
+                ev[0].record()
+            iq.iq_choice_search(d, self.w, self.hess, self.cand, picks=self.picks, payload=self.payload)
+            if ev is not None:
+                ev[1].record()
+
+    def e2e_step(self, host):
+        """Same step through the public API from pinned host memory, results read back."""
+        d = self.desc[self.fmt]
+        if self.kind == "decode":
+            self.payload.copy_(host["payload"], non_blocking=True)
+            iq.iq_decode(d, self.payload, torch.bfloat16, out=self.decoded)
+            host["decoded"].copy_(self.decoded, non_blocking=True)
+        elif self.kind == "encode":
+            self.w.copy_(host["w"], non_blocking=True)
+            if self.imp is not None:
+                self.imp.copy_(host["imp"], non_blocking=True)
+            iq.iq_encode(d, self.w, self.imp, out=self.payload, flags=False)
+            iq.iq_decode(d, self.payload, torch.bfloat16, out=self.decoded)
+            host["payload"].copy_(self.payload, non_blocking=True)
+            host["decoded"].copy_(self.decoded, non_blocking=True)
+        else:
+            self.w.copy_(host["w"], non_blocking=True)
+            self.hess.copy_(host["hess"], non_blocking=True)
+            self.step()
+            host["picks"].copy_(self.picks, non_blocking=True)
+            host["payload"].copy_(self.payload, non_blocking=True)
+
+    def host_buffers(self):
+        pin = lambda t: t.to("cpu").pin_memory()  # noqa: E731
+        if self.kind == "decode":
+            h = {"payload": pin(self.payload), "decoded": pin(self.decoded)}
+            h2d, d2h = self.payload.numel(), self.decoded.numel() * 2
+        elif self.kind == "encode":
+            h = {"w": pin(self.w_host), "payload": pin(self.payload), "decoded": pin(self.decoded)}
+            if self.imp is not None:
+                h["imp"] = pin(self.imp_host)
+            h2d = self.w.numel() * 2 + (0 if self.imp is None else self.imp.numel() * 4)
+            d2h = self.payload.numel() + self.decoded.numel() * 2
+        else:
+            h = {"w": pin(self.w_host), "hess": pin(self.hess_host), "picks": pin(self.picks),
+                 "payload": pin(self.payload)}
+            h2d = self.w.numel() * 2 + self.hess.numel() * 4
+            d2h = self.picks.numel() + self.payload.numel()
+        return h, h2d, d2h
+
+
+def decode_roofline(wl: Workload, dev, peaks):
+    """The decoder timed alone on an HBM-sized input: the workload's payload tiled to ~3.5 GB."""
+    if wl.kind not in ("encode", "decode"):
+        return None
+    B = iq.BLOCK_BYTES[wl.fmt]
+    flat = wl.payload.reshape(-1, B)
+    reps = max(1, (6 << 20) // flat.shape[0])
+    big = flat.repeat(reps, 1)
+    out = torch.empty((big.shape[0], 256), dtype=torch.bfloat16, device=dev)
+    d = wl.desc[wl.fmt]
+    for _ in range(3):
+        iq.iq_decode(d, big, torch.bfloat16, out=out)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    times = []
+    for _ in range(10):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        iq.iq_decode(d, big, torch.bfloat16, out=out)
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e))
+    ms = statistics.median(times)
+    nbytes = big.shape[0] * (B + 512)
+    gbs = nbytes / ms / 1e6
+    del big, out, flush
+    return {"kernel": "decode_kernel (bf16 out)", "blocks": int(flat.shape[0] * reps), "bytes_per_launch": nbytes,
+            "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+            "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "traffic": kernel_traffic("decode_kernel")}
+
+
+# ------------------------------------------------------------------------------------ oracle arm
+
+def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None):
+    """Oracle encode + decode on the first rows of the workload, sized to ~budget_s of wall time."""
+    import oracle
+    if name == "choice_iq2xs_4096x4096":
+        wl = synth.workload_choice_iq2xs()
+        w, hess = wl["w"], wl["hess"].numpy()
+        g = synth.iq2xs_grid()
+        imp = oracle.sqrt_diag(hess)
+
+        def run(r):
+            cand, _ = oracle.encode("iq2_xs", g, iq.DEFAULT_ANCHOR["iq2_xs"], w[:r], importance=imp, every_choice=True)
+            oracle.choice_search("iq2_xs", g, w[:r], hess, cand)
+        cols = w.shape[1]
+    else:
+        if name == "iq1s_moe_256x1536x4096":
+            w, imp = synth.normal_bf16((1536, 4096), 0.02, 1004), synth.lognormal((256, 4096), 3004)[0]
+            fmt = "iq1_s"
+        else:
+            wl = {"iq1s_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
+                  "iq1s_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
+                  "iq2xs_8192x4096": synth.workload_iq2xs_8192x4096,
+                  "iq1s_64x256": synth.workload_iq1s_64x256}[name]()
+            w, imp, fmt = wl["w"], wl["importance"], wl["fmt"]
+        g = synth.iq1s_grid() if fmt == "iq1_s" else synth.iq2xs_grid()
+
+        def run(r):
+            p, _ = oracle.encode(fmt, g, iq.DEFAULT_ANCHOR[fmt], w[:r], importance=imp)
+            oracle.decode(fmt, g, p)
+        cols = w.shape[1]
+    total_rows = w.shape[0]
+    if rows_hint is None:
+        t0 = time.perf_counter()
+        run(1)
+        t1 = time.perf_counter() - t0
+        rows = int(max(1, min(total_rows, budget_s / max(t1, 1e-6))))
+    else:
+        rows = rows_hint
+    t0 = time.perf_counter()
+    run(rows)
+    dt = time.perf_counter() - t0
+    return rows * cols / dt / 1e6, rows, cols, dt, oracle.threads(), run
+
+
+def reference_arm(args, n_gpus, config):
+    import oracle
+    rate, rows, cols, dt, cores, run = oracle_sample_rate(args.workload, budget_s=1.0)
+    # per step: a bounded sample sized so that warm-up + timed steps take about 90 s in all
+    per_row = dt / rows
+    rows = int(max(1, min(rows * 50, 90.0 / (args.steps + args.warmup) / per_row)))
+    for _ in range(args.warmup):
+        run(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run(rows)
+    dt = time.perf_counter() - t0
+    value = args.steps * rows * cols / dt / 1e6
+    sample = f"first {rows} rows x {cols} cols of the workload per step (encode + decode on the host cores)"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": n_gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default="iq1s_4096x4096_weighted")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks = load_peaks()
+    config = {"workload": args.workload, "l2": "flushed before every step (256 MiB write, outside the events)",
+              "parallelism": f"replicas x{world} (independent problems per rank)"}
+
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args, world, config)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    iq.load_library()
+    wl = Workload(args.workload, dev, peaks)
+    config.update({"format": wl.fmt, "shape": list(wl.w.shape), "text": wl.text})
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        wl.step()
+    torch.cuda.synchronize()
+
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dom_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step_ev[i][0].record()
+            wl.step(dom_ev[i])
+            step_ev[i][1].record()
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = sum(s.elapsed_time(e) for s, e in step_ev)
+    dom_ms = [s.elapsed_time(e) for s, e in dom_ev]
+    if dist is not None:
+        t = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    ms_per_step = step_ms / args.steps
+    value = world * wl.units / (ms_per_step / 1e3) / 1e6
+
+    # end to end through the public API from pinned host memory (same stream, events)
+    host, h2d, d2h = wl.host_buffers()
+    for _ in range(2):
+        wl.e2e_step(host)
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 20))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(e2e_steps):
+        wl.e2e_step(host)
+    e.record()
+    torch.cuda.synchronize()
+    e2e_ms = s.elapsed_time(e) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * wl.units / (e2e_ms / 1e3) / 1e6
+
+    dec = decode_roofline(wl, dev, peaks) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    clocks = clk.summary()
+    dom_avg = statistics.mean(dom_ms)
+    if wl.kind == "decode":
+        nbytes = wl.nblocks * (iq.BLOCK_BYTES[wl.fmt] + 512)
+        gbs = nbytes / (dom_avg / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": wl.dominant, "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": kernel_traffic(wl.dominant),
+                "bytes_per_launch": nbytes, "ms_per_launch": round(dom_avg, 4)}
+    else:
+        achieved = wl.ops_per_launch / (dom_avg / 1e3) / 1e12
+        peak = alu_peak_tops(peaks["sm_max_mhz"])
+        roof = {"bound": "alu", "kernel": wl.dominant, "achieved": round(achieved, 3), "peak": round(peak, 3),
+                "unit": "Top/s", "frac": round(achieved / peak, 4), "traffic": kernel_traffic(wl.dominant),
+                "ops_per_launch": wl.ops_per_launch, "ms_per_launch": round(dom_avg, 4),
+                "peak_basis": f"{SMS} SMs x {FP32_LANES} FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (1 op/lane/clock)"}
+        if clocks:
+            roof["frac_at_measured_clock"] = round(achieved / alu_peak_tops(clocks["sm_mhz"]), 4)
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        rate, rows, cols, dt, cores, _ = oracle_sample_rate(args.workload, budget_s=12.0)
+        cpu = {"value": round(rate, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"first {rows} rows x {cols} cols of the workload, encode + decode, {dt:.1f} s wall"}
+
+    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
+            "roofline": roof, "decode": dec, "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks,
+            "peaks": {"source": peaks["source"], "hbm_gbs": peaks["hbm_gbs"]}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -116,7 +116,8 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
     importance: fp32 [cols] or [batch, cols]; choices: uint8 [..., rows, cols/256, G].
     Returns the payload uint8 [(16,) (batch,) rows, cols/256, B]. With raise_on_flags (default)
     the call synchronises and raises on a device-side finding; pass a flags tensor and
-    raise_on_flags=False to stay asynchronous.
+    raise_on_flags=False to stay asynchronous, or flags=False to skip the findings word
+    (invalid blocks are still written as zero payloads).
     """
     lib = load_library()
     fmt = _fmt_of(desc)
@@ -150,9 +151,10 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
         raise IQError(f"out must be a contiguous uint8 tensor of shape {shape}")
     if flags is None:
         flags = torch.empty(1, dtype=torch.int32, device=w.device)
+    flags_ptr = None if flags is False else flags.data_ptr()
     _check(lib.iq_encode(ctypes.byref(desc), w.data_ptr(), batch, rows, cols, ldw, wbs, imp_ptr, imp_bs,
-                         ch_ptr, int(bool(every_choice)), out.data_ptr(), flags.data_ptr(), _stream(stream)))
-    if raise_on_flags:
+                         ch_ptr, int(bool(every_choice)), out.data_ptr(), flags_ptr, _stream(stream)))
+    if raise_on_flags and flags is not False:
         raise_for_flags(flags)
     return out
 

@@ -15,11 +15,13 @@
 //
 // Design (B200): one CTA = 8 warps = 8 rows of one block. The rows run the group steps in
 // lockstep, so each step stages one panel of H (the group's W rows, W x 256 fp32) in shared memory
-// once for all 8 rows; H is read from L2 three times per CTA (step 2 + initial gradient fused in
-// one pass, then one pass per sweep). Inside a warp the 16 choices x W columns of a group are
-// spread as (choice pair, column quad) per lane, so each lane runs 2 x W/4 independent fma chains
-// against broadcast 16-byte panel reads; the gradient is accumulated column-per-thread for all 8
-// rows at once, and a switch updates grad with 16-byte panel reads, 8 columns per lane.
+// once for all 8 rows, double-buffered with cp.async so the next panel streams in while this one
+// is used; H is read from L2 three times per CTA (step 2 + initial gradient fused in one pass,
+// then one pass per sweep). Inside a warp the 16 choices x W columns of a group are spread as
+// (choice pair, column quad) per lane: a lane keeps its two choices' W-vectors in registers and
+// runs 2 x W/4 fma chains that share each 16-byte panel read. The gradient is accumulated
+// column-per-thread for all 8 rows at once, and a switch updates grad with 16-byte panel reads,
+// 8 columns per lane. The grid is staged in shared memory for the candidate decodes.
 #include "iq_device.cuh"
 #include "iq_kernels.h"
 
@@ -34,12 +36,14 @@ struct Cfg {
     static constexpr int W = kBlock / G;                        // columns per choice group
     static constexpr int Q = W / 4;                             // columns per lane (quad split)
     static constexpr int B = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : kIq2xsBytes;
+    static constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : kIq2xsEntries;
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
-    static constexpr int DSTR = W + 1;                          // padded row of Dg
+    static constexpr int DSTR = W + 4;                          // padded row of Dg (16-byte rows)
     // shared memory layout (bytes)
-    static constexpr int oHp = 0;                               // float [W][256]
-    static constexpr int oCurT = oHp + W * kBlock * 4;          // float [256][kRows]
-    static constexpr int oRows = oCurT + kBlock * kRows * 4;    // per-row records
+    static constexpr int oHp = 0;                               // float [2][W][256], double buffer
+    static constexpr int oCurT = oHp + 2 * W * kBlock * 4;      // float [256][kRows]
+    static constexpr int oGrid = oCurT + kBlock * kRows * 4;    // int2 [E]
+    static constexpr int oRows = oGrid + E * 8;                 // per-row records
     static constexpr int rX = 0;                                // float [256]
     static constexpr int rCur = rX + kBlock * 4;                // float [256]
     static constexpr int rGrad = rCur + kBlock * 4;             // float [256]
@@ -51,8 +55,8 @@ struct Cfg {
     static constexpr int smem = oRows + kRows * rBytes;
 };
 
-__device__ __forceinline__ void grid_row(const int8_t* grid, int idx, float g[8]) {
-    const int2 raw = __ldg(reinterpret_cast<const int2*>(grid) + idx);
+__device__ __forceinline__ void grid_row(const int2* sgrid, int idx, float g[8]) {
+    const int2 raw = sgrid[idx];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
         g[j] = static_cast<float>(static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF));
@@ -61,7 +65,7 @@ __device__ __forceinline__ void grid_row(const int8_t* grid, int idx, float g[8]
 // Dg[c][k] = x[gW + k] - decode(candidate c)[gW + k] for all 16 c, k < W. Lane: c = lane / 2,
 // half = lane & 1 decodes W/2 columns.
 template <int FMT>
-__device__ __forceinline__ void decode_group(const uint8_t* cand, const float* x, float* Dg, const int8_t* grid,
+__device__ __forceinline__ void decode_group(const uint8_t* cand, const float* x, float* Dg, const int2* grid,
                                              int g, int lane) {
     using C = Cfg<FMT>;
     const int c = lane >> 1, half = lane & 1;
@@ -130,13 +134,48 @@ __device__ __forceinline__ void warp_argmin(float v0, int c0, float v1, int c1, 
     cbest = c;
 }
 
+template <int N>
+__device__ __forceinline__ void load_vec(const float* src, float v[N]) {
+#pragma unroll
+    for (int t = 0; t < N / 4; ++t) {
+        const float4 a = reinterpret_cast<const float4*>(src)[t];
+        v[4 * t] = a.x; v[4 * t + 1] = a.y; v[4 * t + 2] = a.z; v[4 * t + 3] = a.w;
+    }
+}
+
+// v_h[t] = sum over k < W (fma chain, k ascending) of Hp[k][col0 + t] * a_h[k], for two vectors.
+template <int W, int Q>
+__device__ __forceinline__ void group_matvec2(const float* Hp, int col0, const float a0[W], const float a1[W],
+                                              float v0[Q], float v1[Q]) {
+    float h[Q];
+    load_vec<Q>(Hp + col0, h);
+#pragma unroll
+    for (int t = 0; t < Q; ++t) { v0[t] = __fmul_rn(h[t], a0[0]); v1[t] = __fmul_rn(h[t], a1[0]); }
+#pragma unroll
+    for (int k = 1; k < W; ++k) {
+        load_vec<Q>(Hp + k * kBlock + col0, h);
+#pragma unroll
+        for (int t = 0; t < Q; ++t) {
+            v0[t] = __fmaf_rn(h[t], a0[k], v0[t]);
+            v1[t] = __fmaf_rn(h[t], a1[k], v1[t]);
+        }
+    }
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 template <int FMT>
 __global__ void __launch_bounds__(kRows * 32) choice_search_kernel(const ChoiceParams p) {
     using C = Cfg<FMT>;
     constexpr int W = C::W, Q = C::Q, G = C::G;
     extern __shared__ __align__(16) char smem[];
-    float* Hp = reinterpret_cast<float*>(smem + C::oHp);
     float* curT = reinterpret_cast<float*>(smem + C::oCurT);
+    int2* sgrid = reinterpret_cast<int2*>(smem + C::oGrid);
 
     const int64_t row_tiles = (p.rows + kRows - 1) / kRows;
     const int64_t blk = blockIdx.x / row_tiles;
@@ -154,7 +193,19 @@ __global__ void __launch_bounds__(kRows * 32) choice_search_kernel(const ChoiceP
     uint8_t* cand = reinterpret_cast<uint8_t*>(rec + C::rCand);
     const float* H = p.hess + blk * kBlock * kBlock;
 
-    // ---- stage the row: x (fp32) and the 16 candidate payloads
+    // H panels (the W rows of one choice group) stream through a double buffer: step p of the
+    // 3G group steps (step 2, then two sweeps) uses panel p % G from buffer p & 1.
+    auto panel = [&](int step) { return reinterpret_cast<float*>(smem + C::oHp + (step & 1) * W * kBlock * 4); };
+    auto prefetch = [&](int step) {
+        const char* src = reinterpret_cast<const char*>(H + (step % G) * W * kBlock);
+        char* dst = reinterpret_cast<char*>(panel(step));
+        for (int i = threadIdx.x; i < W * kBlock / 4; i += blockDim.x) cp_async16(dst + 16 * i, src + 16 * i);
+        cp_async_commit();
+    };
+    prefetch(0);
+
+    // ---- stage the grid, the row's x (fp32) and its 16 candidate payloads
+    for (int q = threadIdx.x; q < C::E; q += blockDim.x) sgrid[q] = __ldg(reinterpret_cast<const int2*>(p.grid) + q);
     if (active) {
         float xv[8];
         unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(p.w + row * p.ldw + blk * kBlock) + lane), xv);
@@ -172,48 +223,36 @@ __global__ void __launch_bounds__(kRows * 32) choice_search_kernel(const ChoiceP
     } else {
         for (int i = lane; i < kBlock; i += 32) curT[i * kRows + warp] = 0.0f;
     }
-    __syncwarp();
-
-    auto load_panel = [&](int g) {
-        __syncthreads();  // everyone is done with the previous panel
-        const float4* src = reinterpret_cast<const float4*>(H + g * W * kBlock);
-        float4* dst = reinterpret_cast<float4*>(Hp);
-        for (int i = threadIdx.x; i < W * kBlock / 4; i += blockDim.x) dst[i] = __ldg(src + i);
-        __syncthreads();
-    };
 
     const int cp = lane >> 2, iq = lane & 3;
     const int c0 = 2 * cp, c1 = 2 * cp + 1;
+    const float* D0 = Dg + c0 * C::DSTR;
+    const float* D1 = Dg + c1 * C::DSTR;
 
     // ---- step 2 (own diagonal block) fused with the initial gradient grad = H Delta
     float gacc[kRows];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) gacc[r] = 0.0f;
     for (int g = 0; g < G; ++g) {
-        load_panel(g);
+        cp_async_wait_all();
+        __syncthreads();  // panel g has landed; every thread is done with the other buffer
+        prefetch(g + 1);
+        const float* Hp = panel(g);
         if (active) {
-            decode_group<FMT>(cand, x, Dg, p.grid, g, lane);
+            decode_group<FMT>(cand, x, Dg, sgrid, g, lane);
             __syncwarp();
-            float sc[2];
+            float a0[W], a1[W], v0[Q], v1[Q], e0[Q], e1[Q];
+            load_vec<W>(D0, a0);
+            load_vec<W>(D1, a1);
+            group_matvec2<W, Q>(Hp, g * W + iq * Q, a0, a1, v0, v1);
+            load_vec<Q>(D0 + iq * Q, e0);
+            load_vec<Q>(D1 + iq * Q, e1);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float* D = Dg + (h ? c1 : c0) * C::DSTR;
-                float v[Q];
-#pragma unroll
-                for (int t = 0; t < Q; ++t) v[t] = __fmul_rn(Hp[g * W + iq * Q + t], D[0]);
-#pragma unroll 4
-                for (int k = 1; k < W; ++k) {
-                    const float dk = D[k];
-#pragma unroll
-                    for (int t = 0; t < Q; ++t) v[t] = __fmaf_rn(Hp[k * kBlock + g * W + iq * Q + t], dk, v[t]);
-                }
-#pragma unroll
-                for (int t = 0; t < Q; ++t) v[t] = __fmul_rn(D[iq * Q + t], v[t]);
-                sc[h] = quad_tree<Q>(v);
-            }
+            for (int t = 0; t < Q; ++t) { v0[t] = __fmul_rn(e0[t], v0[t]); v1[t] = __fmul_rn(e1[t], v1[t]); }
+            const float s0 = quad_tree<Q>(v0), s1 = quad_tree<Q>(v1);
             float best;
             int cstar;
-            warp_argmin(sc[0], c0, sc[1], c1, best, cstar);
+            warp_argmin(s0, c0, s1, c1, best, cstar);
             if (lane < W) {
                 const float dv = Dg[cstar * C::DSTR + lane];
                 cur[g * W + lane] = dv;
@@ -225,7 +264,7 @@ __global__ void __launch_bounds__(kRows * 32) choice_search_kernel(const ChoiceP
         // grad_i += H[k][i] cur_k over this group's k, for all rows (thread = column i)
         {
             const int i = threadIdx.x;
-#pragma unroll 2
+#pragma unroll 4
             for (int k = 0; k < W; ++k) {
                 const float h = Hp[k * kBlock + i];
                 const float4 ca = *reinterpret_cast<const float4*>(curT + (g * W + k) * kRows);
@@ -251,67 +290,73 @@ __global__ void __launch_bounds__(kRows * 32) choice_search_kernel(const ChoiceP
     }
 
     // ---- step 3: two sweeps over the groups
-    for (int sweep = 0; sweep < 2; ++sweep) {
-        for (int g = 0; g < G; ++g) {
-            load_panel(g);
-            if (!active) continue;
-            decode_group<FMT>(cand, x, Dg, p.grid, g, lane);
-            __syncwarp();
-            float gain[2];
+    for (int step = G; step < 3 * G; ++step) {
+        const int g = step % G;
+        cp_async_wait_all();
+        __syncthreads();
+        if (step + 1 < 3 * G) prefetch(step + 1);
+        const float* Hp = panel(step);
+        if (!active) continue;
+        decode_group<FMT>(cand, x, Dg, sgrid, g, lane);
+        __syncwarp();
+        float u0[W], u1[W], v0[Q], v1[Q];
+        {
+            float cg[W];
+            load_vec<W>(cur + g * W, cg);
+            load_vec<W>(D0, u0);
+            load_vec<W>(D1, u1);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float* D = Dg + (h ? c1 : c0) * C::DSTR;
-                float u[Q], pt[Q], v[Q];
-#pragma unroll
-                for (int t = 0; t < Q; ++t) {
-                    u[t] = __fsub_rn(D[iq * Q + t], cur[g * W + iq * Q + t]);
-                    pt[t] = __fmul_rn(u[t], grad[g * W + iq * Q + t]);
-                }
-                const float t1 = quad_tree<Q>(pt);
-                {
-                    const float u0 = __fsub_rn(D[0], cur[g * W]);
-#pragma unroll
-                    for (int t = 0; t < Q; ++t) v[t] = __fmul_rn(Hp[g * W + iq * Q + t], u0);
-                }
-#pragma unroll 4
-                for (int k = 1; k < W; ++k) {
-                    const float uk = __fsub_rn(D[k], cur[g * W + k]);
-#pragma unroll
-                    for (int t = 0; t < Q; ++t) v[t] = __fmaf_rn(Hp[k * kBlock + g * W + iq * Q + t], uk, v[t]);
-                }
-#pragma unroll
-                for (int t = 0; t < Q; ++t) v[t] = __fmul_rn(u[t], v[t]);
-                const float t2 = quad_tree<Q>(v);
-                gain[h] = __fmaf_rn(2.0f, t1, t2);
-            }
-            float best;
-            int cstar;
-            warp_argmin(gain[0], c0, gain[1], c1, best, cstar);
-            if (best < 0.0f) {
-                if (lane < W) ustar[lane] = __fsub_rn(Dg[cstar * C::DSTR + lane], cur[g * W + lane]);
-                __syncwarp();
-                // grad[i] += sum_k H[k][i] u_k (fma chain over the group's k), 8 columns per lane
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int i0 = half * 128 + 4 * lane;
-                    float4 acc = *reinterpret_cast<const float4*>(grad + i0);
-#pragma unroll 4
-                    for (int k = 0; k < W; ++k) {
-                        const float uk = ustar[k];
-                        const float4 hv = *reinterpret_cast<const float4*>(Hp + k * kBlock + i0);
-                        acc.x = __fmaf_rn(hv.x, uk, acc.x);
-                        acc.y = __fmaf_rn(hv.y, uk, acc.y);
-                        acc.z = __fmaf_rn(hv.z, uk, acc.z);
-                        acc.w = __fmaf_rn(hv.w, uk, acc.w);
-                    }
-                    *reinterpret_cast<float4*>(grad + i0) = acc;
-                }
-                __syncwarp();
-                if (lane < W) cur[g * W + lane] = Dg[cstar * C::DSTR + lane];
-                if (lane == 0) pick[g] = cstar;
-            }
-            __syncwarp();
+            for (int k = 0; k < W; ++k) { u0[k] = __fsub_rn(u0[k], cg[k]); u1[k] = __fsub_rn(u1[k], cg[k]); }
         }
+        group_matvec2<W, Q>(Hp, g * W + iq * Q, u0, u1, v0, v1);
+        float gain0, gain1;
+        {
+            float cq[Q], e0[Q], e1[Q], gq[Q], p0[Q], p1[Q];
+            load_vec<Q>(cur + g * W + iq * Q, cq);
+            load_vec<Q>(D0 + iq * Q, e0);
+            load_vec<Q>(D1 + iq * Q, e1);
+            load_vec<Q>(grad + g * W + iq * Q, gq);
+#pragma unroll
+            for (int t = 0; t < Q; ++t) {
+                e0[t] = __fsub_rn(e0[t], cq[t]);  // u_i of this lane's columns
+                e1[t] = __fsub_rn(e1[t], cq[t]);
+                p0[t] = __fmul_rn(e0[t], gq[t]);
+                p1[t] = __fmul_rn(e1[t], gq[t]);
+                v0[t] = __fmul_rn(e0[t], v0[t]);
+                v1[t] = __fmul_rn(e1[t], v1[t]);
+            }
+            const float t10 = quad_tree<Q>(p0), t11 = quad_tree<Q>(p1);
+            const float t20 = quad_tree<Q>(v0), t21 = quad_tree<Q>(v1);
+            gain0 = __fmaf_rn(2.0f, t10, t20);
+            gain1 = __fmaf_rn(2.0f, t11, t21);
+        }
+        float best;
+        int cstar;
+        warp_argmin(gain0, c0, gain1, c1, best, cstar);
+        if (best < 0.0f) {
+            if (lane < W) ustar[lane] = __fsub_rn(Dg[cstar * C::DSTR + lane], cur[g * W + lane]);
+            __syncwarp();
+            // grad[i] += sum_k H[k][i] u_k (fma chain over the group's k), 8 columns per lane
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int i0 = half * 128 + 4 * lane;
+                float4 acc = *reinterpret_cast<const float4*>(grad + i0);
+#pragma unroll 4
+                for (int k = 0; k < W; ++k) {
+                    const float uk = ustar[k];
+                    const float4 hv = *reinterpret_cast<const float4*>(Hp + k * kBlock + i0);
+                    acc.x = __fmaf_rn(hv.x, uk, acc.x);
+                    acc.y = __fmaf_rn(hv.y, uk, acc.y);
+                    acc.z = __fmaf_rn(hv.z, uk, acc.z);
+                    acc.w = __fmaf_rn(hv.w, uk, acc.w);
+                }
+                *reinterpret_cast<float4*>(grad + i0) = acc;
+            }
+            __syncwarp();
+            if (lane < W) cur[g * W + lane] = Dg[cstar * C::DSTR + lane];
+            if (lane == 0) pick[g] = cstar;
+        }
+        __syncwarp();
     }
 
     // ---- step 4: picks and the payload assembled from the picked candidates

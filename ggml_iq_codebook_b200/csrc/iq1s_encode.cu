@@ -20,8 +20,8 @@
 // shared-memory read, and each lane then reads its own group's nibble tables (S(w), S(T) for the
 // 16 low and 16 high nibble values, 8 KiB per warp, conflict-free rows). The argmin keeps only
 // running minima (fminf) in registers plus the chunk of K entries where each choice's minimum
-// first appeared; the winning entry index is recovered afterwards by rescanning that one chunk
-// with the identical arithmetic. Persistent CTAs walk the blocks with a static stride: every
+// first appeared (two candidates fold into one three-input min); the winning entry index is
+// recovered afterwards by rescanning that one chunk with the identical arithmetic. Persistent CTAs walk the blocks with a static stride: every
 // block costs the same, so no work queue (and no scratch memory) is needed.
 #include "iq_device.cuh"
 #include "iq_kernels.h"
@@ -57,7 +57,7 @@ __device__ __forceinline__ Terms entry_terms(const char* smem, uint32_t lane_bas
 }
 
 __device__ __forceinline__ void write_zero_block(uint8_t* out, int lane) {
-    if (lane < kIq1sBytes / 2) reinterpret_cast<uint16_t*>(out)[lane] = 0;
+    for (int i = lane; i < kIq1sBytes / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
 }
 
 // Pack one block: lane = group, idx = its entry, c = its sub-block's choice.
@@ -201,20 +201,22 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
         for (int ch = 0; ch < kIq1sEntries / K; ++ch) {
             float cm[kChoices];
             {
-                const Terms tm = entry_terms(smem, lane_base, sgrid[ch * K], W, Tall);
+                const Terms ta = entry_terms(smem, lane_base, sgrid[ch * K], W, Tall);
+                const Terms tb = entry_terms(smem, lane_base, sgrid[ch * K + 1], W, Tall);
 #pragma unroll
                 for (int ls = 0; ls < 8; ++ls) {
-                    cm[ls] = __fmaf_rn(s[ls], tm.Ap, tm.Cp);
-                    cm[8 + ls] = __fmaf_rn(s[ls], tm.An, tm.Cn);
+                    cm[ls] = fminf(__fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
+                    cm[8 + ls] = fminf(__fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
                 }
             }
-#pragma unroll 4
-            for (int q = ch * K + 1; q < ch * K + K; ++q) {
-                const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+#pragma unroll 2
+            for (int q = ch * K + 2; q < ch * K + K; q += 2) {
+                const Terms ta = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+                const Terms tb = entry_terms(smem, lane_base, sgrid[q + 1], W, Tall);
 #pragma unroll
                 for (int ls = 0; ls < 8; ++ls) {
-                    cm[ls] = fminf(cm[ls], __fmaf_rn(s[ls], tm.Ap, tm.Cp));
-                    cm[8 + ls] = fminf(cm[8 + ls], __fmaf_rn(s[ls], tm.An, tm.Cn));
+                    cm[ls] = min3f(cm[ls], __fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
+                    cm[8 + ls] = min3f(cm[8 + ls], __fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
                 }
             }
 #pragma unroll
@@ -279,7 +281,7 @@ cudaError_t launch_iq1s_encode(const EncodeParams& p, int mode, int num_sms, cud
     switch (mode) {
         case kSearch: return launch_mode<kSearch, 32>(p, num_sms, s);
         case kFixed: return launch_mode<kFixed, 32>(p, num_sms, s);
-        default: return launch_mode<kEvery, 16>(p, num_sms, s);
+        default: return launch_mode<kEvery, 8>(p, num_sms, s);
     }
 }
 

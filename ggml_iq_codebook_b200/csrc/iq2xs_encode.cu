@@ -16,7 +16,8 @@
 // Kernel design (B200): one warp per block, one lane per group; the 512-entry loop is warp-uniform
 // and reads each entry's 8 magnitudes and 8 squares (64 B) with broadcast 16-byte shared-memory
 // loads. Argmin bookkeeping as in the IQ1_S kernel: running minima, chunk of first appearance,
-// one-chunk rescan for the index.
+// one-chunk rescan for the index; the rescans, whose entries differ from lane to lane, read a
+// packed 8-byte copy of the grid instead of the 64-byte float rows.
 #include "iq_device.cuh"
 #include "iq_kernels.h"
 
@@ -24,7 +25,8 @@ namespace iqk {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kSmemBytes = kIq2xsEntries * 16 * 4;  // per entry: g[8] then g^2[8] as fp32
+constexpr int kFloatGridBytes = kIq2xsEntries * 16 * 4;  // per entry: g[8] then g^2[8] as fp32
+constexpr int kSmemBytes = kFloatGridBytes + kIq2xsEntries * 8;  // + the packed int8 grid
 
 struct Entry {
     float g[8], gg[8];
@@ -36,6 +38,17 @@ __device__ __forceinline__ void load_entry(const float4* sg, int q, Entry& en) {
     en.g[4] = b.x; en.g[5] = b.y; en.g[6] = b.z; en.g[7] = b.w;
     en.gg[0] = c.x; en.gg[1] = c.y; en.gg[2] = c.z; en.gg[3] = c.w;
     en.gg[4] = d.x; en.gg[5] = d.y; en.gg[6] = d.z; en.gg[7] = d.w;
+}
+
+// The same entry rebuilt from the packed int8 grid (one 8-byte read): the rescans of single
+// chunks read entries at lane-dependent addresses, where 8 bytes beat 64.
+__device__ __forceinline__ void load_entry_packed(const int2* sp, int q, Entry& en) {
+    const int2 raw = sp[q];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        en.g[j] = static_cast<float>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
+        en.gg[j] = __fmul_rn(en.g[j], en.g[j]);
+    }
 }
 
 __device__ __forceinline__ void entry_AB(const Entry& en, const float w[8], const float V[8], float& A,
@@ -50,7 +63,7 @@ __device__ __forceinline__ void entry_AB(const Entry& en, const float w[8], cons
 }
 
 __device__ __forceinline__ void write_zero_block(uint8_t* out, int lane) {
-    if (lane < kIq2xsBytes / 2) reinterpret_cast<uint16_t*>(out)[lane] = 0;
+    for (int i = lane; i < kIq2xsBytes / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
 }
 
 // lane = group: code = idx | sign7 << 9; ls = its sub-block's local scale.
@@ -68,10 +81,12 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
     extern __shared__ __align__(16) char smem[];
     float* sgf = reinterpret_cast<float*>(smem);
     const float4* sg = reinterpret_cast<const float4*>(smem);
+    int2* sgp = reinterpret_cast<int2*>(smem + kFloatGridBytes);
 
     bool bad = false;
     for (int q = threadIdx.x; q < kIq2xsEntries; q += blockDim.x) {
         const int2 raw = __ldg(reinterpret_cast<const int2*>(p.grid) + q);
+        sgp[q] = raw;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
@@ -186,21 +201,26 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
         for (int ch = 0; ch < kIq2xsEntries / K; ++ch) {
             float cm[kChoices];
             {
-                Entry en;
-                load_entry(sg, ch * K, en);
-                float A, B;
-                entry_AB(en, w, V, A, B);
+                Entry ea, eb;
+                load_entry(sg, ch * K, ea);
+                load_entry(sg, ch * K + 1, eb);
+                float Aa, Ba, Ab, Bb;
+                entry_AB(ea, w, V, Aa, Ba);
+                entry_AB(eb, w, V, Ab, Bb);
 #pragma unroll
-                for (int c = 0; c < kChoices; ++c) cm[c] = __fmaf_rn(s[c], A, B);
+                for (int c = 0; c < kChoices; ++c) cm[c] = fminf(__fmaf_rn(s[c], Aa, Ba), __fmaf_rn(s[c], Ab, Bb));
             }
-#pragma unroll 2
-            for (int q = ch * K + 1; q < ch * K + K; ++q) {
-                Entry en;
-                load_entry(sg, q, en);
-                float A, B;
-                entry_AB(en, w, V, A, B);
+#pragma unroll 1
+            for (int q = ch * K + 2; q < ch * K + K; q += 2) {
+                Entry ea, eb;
+                load_entry(sg, q, ea);
+                load_entry(sg, q + 1, eb);
+                float Aa, Ba, Ab, Bb;
+                entry_AB(ea, w, V, Aa, Ba);
+                entry_AB(eb, w, V, Ab, Bb);
 #pragma unroll
-                for (int c = 0; c < kChoices; ++c) cm[c] = fminf(cm[c], __fmaf_rn(s[c], A, B));
+                for (int c = 0; c < kChoices; ++c)
+                    cm[c] = min3f(cm[c], __fmaf_rn(s[c], Aa, Ba), __fmaf_rn(s[c], Ab, Bb));
             }
 #pragma unroll
             for (int c = 0; c < kChoices; ++c) {
@@ -216,7 +236,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
             if (!(target < INFINITY)) return 0;
             for (int q = ch * K; q < ch * K + K; ++q) {
                 Entry en;
-                load_entry(sg, q, en);
+                load_entry_packed(sgp, q, en);
                 float A, B;
                 entry_AB(en, w, V, A, B);
                 if (__fmaf_rn(sv, A, B) == target) return q;
@@ -259,7 +279,7 @@ cudaError_t launch_iq2xs_encode(const EncodeParams& p, int mode, int num_sms, cu
     switch (mode) {
         case kSearch: return launch_mode<kSearch, 32>(p, num_sms, s);
         case kFixed: return launch_mode<kFixed, 32>(p, num_sms, s);
-        default: return launch_mode<kEvery, 16>(p, num_sms, s);
+        default: return launch_mode<kEvery, 8>(p, num_sms, s);
     }
 }
 

@@ -112,6 +112,8 @@ int32_t iq_num_choices(int32_t fmt);
  *          nibble of byte 66+i.
  * Value of a weight: IQ1_S d (2 ls + 1)(q + delta); IQ2_XS d (2 ls + 1) g sign.
  * amax == 0, or d rounding to fp16 zero, gives the all-zero payload ([#2450]).
+ * Alignment: w and importance 16-byte aligned, ldw and w_batch_stride multiples of 8 elements,
+ * imp_batch_stride a multiple of 4, payload 2-byte aligned, grid 16-byte aligned (IQ_EINVAL).
  */
 iq_status iq_encode(const iq_desc *desc, const uint16_t *w, int64_t batch, int64_t rows, int64_t cols,
                     int64_t ldw, int64_t w_batch_stride, const float *importance,
@@ -121,6 +123,7 @@ iq_status iq_encode(const iq_desc *desc, const uint16_t *w, int64_t batch, int64
 /*
  * Decode nblocks contiguous payload blocks into [nblocks][256] values, fp32 (exact) or bf16
  * (round to nearest even of the exact value). Output is independent of how blocks are chunked.
+ * payload must be 2-byte aligned and out 16-byte aligned (IQ_EINVAL otherwise).
  */
 iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks, int32_t out_dtype,
                     void *out, cudaStream_t stream);
