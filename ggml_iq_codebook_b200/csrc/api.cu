@@ -114,7 +114,7 @@ iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks
     if (payload == nullptr || out == nullptr) return IQ_EINVAL;
     if (nblocks <= 0) return IQ_ESHAPE;
     if (out_dtype != IQ_OUT_F32 && out_dtype != IQ_OUT_BF16) return IQ_EINVAL;
-    if (!aligned(out, 16) || !aligned(payload, 2)) return IQ_EINVAL;
+    if (!aligned(out, 32) || !aligned(payload, 2)) return IQ_EINVAL;
     int sms = 0;
     if ((st = device_sms(&sms)) != IQ_OK) return st;
     iqk::DecodeParams p;

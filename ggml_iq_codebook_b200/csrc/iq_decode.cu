@@ -9,147 +9,200 @@
 // output is its round-to-nearest-even. Each block decodes independently, so the output does not
 // depend on how a caller chunks the blocks.
 //
-// Design: one warp per block, one lane per 8-weight group. The warp reads the block's payload as
-// 16-bit words (one per lane, coalesced into one or two sectors) and hands each lane its fields
-// with warp shuffles. Each warp works on 8 blocks at a time and issues the payload loads of its
-// next 8 blocks before decoding the current ones, so HBM latency overlaps the work; the grid
-// (16 KiB / 4 KiB) is staged once per CTA in shared memory, so no global load depends on another.
-// Each lane writes its 8 outputs with one 16-byte (bf16) or two 16-byte (fp32) streaming stores:
-// a warp writes 512 or 1024 contiguous bytes per block.
+// Design: persistent CTAs walk tiles of 256 blocks. A tile's payload bytes (12.5 / 18.5 KiB)
+// stream into shared memory with 16-byte cp.async copies, double-buffered, so the next tile's
+// reads are in flight while this one is decoded and no warp waits on its own small global loads.
+// A half-warp decodes one block, two adjacent 8-weight groups per lane, reading its fields from
+// the staged bytes; the grid is staged once per CTA as 16-bit element codes (4 KiB / 1 KiB), and
+// outputs are picked from a lane's precomputed products (no int-to-float conversions, which
+// throttle the MIO queue). Each lane writes its 16 outputs with 32-byte streaming stores
+// (st.global.v8): one for bf16, two for fp32.
 #include "iq_device.cuh"
 #include "iq_kernels.h"
 
 namespace iqk {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kUnroll = 8;  // blocks per warp per iteration (and as many prefetched)
+#ifndef IQ_DECODE_MIN_CTAS
+#define IQ_DECODE_MIN_CTAS 1  // launch-bounds occupancy hint (CTAs per SM)
+#endif
 
+#ifndef IQ_DECODE_TILE
+#define IQ_DECODE_TILE 256  // blocks per staged payload tile
+#endif
+#ifndef IQ_DECODE_CTAS
+#define IQ_DECODE_CTAS 5  // persistent CTAs per SM
+#endif
+
+constexpr int kThreads = 256;
+constexpr int kTileBlocks = IQ_DECODE_TILE;
+constexpr int kCtasPerSm = IQ_DECODE_CTAS;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
+}
+
+__device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                             uint32_t f, uint32_t g, uint32_t h) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a), "r"(b), "r"(c),
+                 "r"(d), "r"(e), "r"(f), "r"(g), "r"(h)
+                 : "memory");
+}
+
+// Store 16 consecutive outputs (two groups) starting at output element 8 * group.
 template <bool BF16>
-__device__ __forceinline__ void store8(void* out, int64_t group, const float v[8]) {
+__device__ __forceinline__ void store16(void* out, int64_t group, const float v[16]) {
     if (BF16) {
-        uint4 o;
-        o.x = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[0]))) |
-              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[1]))) << 16);
-        o.y = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[2]))) |
-              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[3]))) << 16);
-        o.z = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[4]))) |
-              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[5]))) << 16);
-        o.w = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[6]))) |
-              (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v[7]))) << 16);
-        __stcs(reinterpret_cast<uint4*>(out) + group, o);
+        uint32_t w[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) w[t] = pack_bf16x2(v[2 * t], v[2 * t + 1]);
+        st_global_v8(reinterpret_cast<uint4*>(out) + group, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
     } else {
         float4* o = reinterpret_cast<float4*>(out) + 2 * group;
-        __stcs(o, make_float4(v[0], v[1], v[2], v[3]));
-        __stcs(o + 1, make_float4(v[4], v[5], v[6], v[7]));
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            st_global_v8(o + 2 * h, __float_as_uint(v[8 * h]), __float_as_uint(v[8 * h + 1]),
+                         __float_as_uint(v[8 * h + 2]), __float_as_uint(v[8 * h + 3]), __float_as_uint(v[8 * h + 4]),
+                         __float_as_uint(v[8 * h + 5]), __float_as_uint(v[8 * h + 6]), __float_as_uint(v[8 * h + 7]));
     }
 }
 
-__device__ __forceinline__ void grid_row(const int2* grid, int idx, float g[8]) {
-    const int2 raw = grid[idx];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        g[j] = static_cast<float>(static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF));
-}
 
-// Fields of this lane's group from the block's 16-bit words (v0: word `lane`, v1: word 32+lane).
-template <int FMT>
-__device__ __forceinline__ void group_fields(uint32_t v0, uint32_t v1, int lane, float& s, float& delta,
-                                             int& idx, uint32_t& neg) {
-    const float d = half_bits_to_f32(__shfl_sync(0xffffffffu, v0, 0));
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// A half-warp decodes one block from its staged payload bytes `pb` (2-byte aligned); lane
+// h = lane & 15 decodes groups 2h and 2h + 1. No int-to-float conversion on the way: a lane
+// forms the few products a group can take (IQ1_S: s (q + delta) for q in {-1, 0, 1}; IQ2_XS:
+// s g for g in {1, 3, 5, 7}), each rounded exactly as the direct formula rounds it, and picks
+// per element from the staged grid codes.
+template <int FMT, bool BF16>
+__device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint16_t* sgrid, void* out, int64_t b) {
+    const uint16_t* pw = reinterpret_cast<const uint16_t*>(pb);
+    float v[16];
+    const float d = half_bits_to_f32(pw[0]);
     if (FMT == IQ_FMT_IQ1_S) {
-        const uint32_t lw = __shfl_sync(0xffffffffu, v0, 1 + (lane >> 1));
-        const uint32_t qh = __shfl_sync(0xffffffffu, v0, 17 + (lane >> 2));
-        const uint32_t low = (lane & 1) ? (lw >> 8) : (lw & 0xFFu);
-        idx = static_cast<int>(low | (((qh >> (3 * (lane & 3))) & 7u) << 8));
-        s = __fmul_rn(d, static_cast<float>(2 * static_cast<int>((qh >> 12) & 7u) + 1));
-        delta = (qh & 0x8000u) ? -0.125f : 0.125f;
-        neg = 0;
-    } else {
-        const uint32_t ca = __shfl_sync(0xffffffffu, v0, lane < 31 ? lane + 1 : 31);
-        const uint32_t cb = __shfl_sync(0xffffffffu, v1, 0);
-        const uint32_t code = lane < 31 ? ca : cb;
-        const uint32_t sw = __shfl_sync(0xffffffffu, v1, 1 + (lane >> 3));  // bytes 66 + 2m, 67 + 2m
-        const uint32_t sc = ((lane >> 2) & 1) ? (sw >> 8) : (sw & 0xFFu);
-        const int ls = static_cast<int>(((lane >> 1) & 1) ? (sc >> 4) : (sc & 15u));
-        s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
-        delta = 0.0f;
-        idx = static_cast<int>(code & 511u);
-        const uint32_t sign7 = code >> 9;
-        neg = sign7 | (static_cast<uint32_t>(__popc(sign7) & 1) << 7);
-    }
-}
-
-template <int WORDS>
-__device__ __forceinline__ void load_words(const uint16_t* words, int64_t b0, int64_t nblocks, int lane,
-                                           uint32_t v0[kUnroll], uint32_t v1[kUnroll]) {
+        const uint32_t lw = pw[1 + h];          // low index bytes of groups 2h, 2h + 1
+        const uint32_t qh = pw[17 + (h >> 1)];  // the sub-block's qh
+        const float s = __fmul_rn(d, static_cast<float>(2 * static_cast<int>((qh >> 12) & 7u) + 1));
+        const float delta = (qh & 0x8000u) ? -0.125f : 0.125f;
+        const float vp = __fmul_rn(s, __fadd_rn(1.0f, delta));   // q = +1
+        const float v0 = __fmul_rn(s, __fadd_rn(0.0f, delta));   // q = 0
+        const float vn = __fmul_rn(s, __fadd_rn(-1.0f, delta));  // q = -1
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-        const int64_t b = b0 + u;
-        v0[u] = 0;
-        v1[u] = 0;
-        if (b < nblocks) {
-            if (lane < WORDS) v0[u] = __ldcs(words + b * WORDS + lane);
-            if (WORDS > 32 && lane < WORDS - 32) v1[u] = __ldcs(words + b * WORDS + 32 + lane);
+        for (int t = 0; t < 2; ++t) {
+            const int grp = 2 * h + t;
+            const int idx = static_cast<int>(((lw >> (8 * t)) & 0xFFu) | (((qh >> (3 * (grp & 3))) & 7u) << 8));
+            const uint32_t m = sgrid[idx];  // bit j: q_j = +1; bit 8 + j: q_j = -1
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[8 * t + j] = ((m >> j) & 1u) ? vp : (((m >> (8 + j)) & 1u) ? vn : v0);
+        }
+    } else {
+        const uint32_t ca = pw[1 + 2 * h], cb = pw[2 + 2 * h];  // codes of groups 2h, 2h + 1
+        const uint32_t sc = pb[66 + (h >> 1)];                   // scales of sub-blocks 2(h/2), +1
+        const int ls = static_cast<int>((h & 1) ? (sc >> 4) : (sc & 15u));
+        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t code = t ? cb : ca;
+            const uint32_t sign7 = code >> 9;
+            const uint32_t neg = sign7 | (static_cast<uint32_t>(__popc(sign7) & 1) << 7);
+            const uint32_t e = sgrid[code & 511u];  // 2 bits per element: g = 2 * bits + 1
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t cj = (e >> (2 * j)) & 3u;
+                const float a = (cj & 2u) ? ((cj & 1u) ? m7 : m5) : ((cj & 1u) ? m3 : m1);
+                v[8 * t + j] = ((neg >> j) & 1u) ? -a : a;
+            }
         }
     }
+    store16<BF16>(out, b * 32 + 2 * h, v);
+}
+
+template <int FMT>
+struct DecodeCfg {
+    static constexpr int BYTES = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : kIq2xsBytes;
+    static constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : kIq2xsEntries;
+    static constexpr int TILE_BYTES = kTileBlocks * BYTES;  // a multiple of 16
+    static constexpr int GRID_BYTES = (E * 2 + 15) / 16 * 16;
+    static constexpr int smem = GRID_BYTES + 2 * TILE_BYTES;
+};
+
+// The grid as 16-bit codes: IQ1_S (+1 mask) | (-1 mask) << 8; IQ2_XS two bits (g - 1) / 2 per
+// element. Values outside the format's alphabet are not representable here.
+template <int FMT>
+__device__ __forceinline__ uint16_t grid_code(int2 raw) {
+    uint32_t c = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
+        if (FMT == IQ_FMT_IQ1_S) c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
+        else c |= (static_cast<uint32_t>((v - 1) >> 1) & 3u) << (2 * j);
+    }
+    return static_cast<uint16_t>(c);
 }
 
 template <int FMT, bool BF16>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
-    constexpr int BYTES = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : kIq2xsBytes;
-    constexpr int WORDS = BYTES / 2;
-    constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : kIq2xsEntries;
-    __shared__ int2 sgrid[E];
-    for (int q = threadIdx.x; q < E; q += kThreads) sgrid[q] = __ldg(reinterpret_cast<const int2*>(p.grid) + q);
-    __syncthreads();
+__global__ void __launch_bounds__(kThreads, IQ_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p) {
+    using C = DecodeCfg<FMT>;
+    extern __shared__ __align__(16) char smem[];
+    uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem);
+    uint8_t* tiles = reinterpret_cast<uint8_t*>(smem + C::GRID_BYTES);
+    for (int q = threadIdx.x; q < C::E; q += kThreads)
+        sgrid[q] = grid_code<FMT>(__ldg(reinterpret_cast<const int2*>(p.grid) + q));
 
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-    const int64_t stride = nwarps * kUnroll;
-    const uint16_t* words = reinterpret_cast<const uint16_t*>(p.payload);
-
-    uint32_t v0[kUnroll], v1[kUnroll];
-    int64_t b0 = warp * kUnroll;
-    load_words<WORDS>(words, b0, p.nblocks, lane, v0, v1);
-    for (; b0 < p.nblocks; b0 += stride) {
-        uint32_t n0[kUnroll], n1[kUnroll];
-        load_words<WORDS>(words, b0 + stride, p.nblocks, lane, n0, n1);  // next batch, in flight
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t b = b0 + u;
-            if (b >= p.nblocks) break;  // warp-uniform
-            float s, delta;
-            int idx;
-            uint32_t neg;
-            group_fields<FMT>(v0[u], v1[u], lane, s, delta, idx, neg);
-            float g[8], v[8];
-            grid_row(sgrid, idx, g);
-            if (FMT == IQ_FMT_IQ1_S) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(s, __fadd_rn(g[j], delta));
+    const int64_t ntiles = (p.nblocks + kTileBlocks - 1) / kTileBlocks;
+    const bool aligned16 = (reinterpret_cast<uintptr_t>(p.payload) & 15u) == 0;
+    // Stage tile t into buffer buf: 16-byte async copies when the tile is whole and aligned,
+    // plain byte copies otherwise (made visible by the barrier before the tile is read).
+    auto stage = [&](int64_t t, int buf) {
+        if (t < ntiles) {
+            const int64_t nb = p.nblocks - t * kTileBlocks < kTileBlocks ? p.nblocks - t * kTileBlocks : kTileBlocks;
+            const int bytes = static_cast<int>(nb) * C::BYTES;
+            const uint8_t* src = p.payload + t * C::TILE_BYTES;
+            uint8_t* dst = tiles + buf * C::TILE_BYTES;
+            if (aligned16 && (bytes & 15) == 0) {
+                for (int i = threadIdx.x; i < bytes / 16; i += kThreads) cp_async16(dst + 16 * i, src + 16 * i);
             } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float a = __fmul_rn(s, g[j]);
-                    v[j] = ((neg >> j) & 1u) ? -a : a;
-                }
+                for (int i = threadIdx.x; i < bytes; i += kThreads) dst[i] = src[i];
             }
-            store8<BF16>(p.out, b * 32 + lane, v);
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) { v0[u] = n0[u]; v1[u] = n1[u]; }
+        cp_async_commit();
+    };
+
+    const int hw = threadIdx.x >> 4, h = threadIdx.x & 15;  // half-warp, lane within it
+    int buf = 0;
+    stage(blockIdx.x, 0);
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, buf ^= 1) {
+        stage(t + gridDim.x, buf ^ 1);  // the next tile streams in while this one is decoded
+        cp_async_wait<1>();
+        __syncthreads();
+        const int64_t nb = p.nblocks - t * kTileBlocks < kTileBlocks ? p.nblocks - t * kTileBlocks : kTileBlocks;
+        const uint8_t* tile = tiles + buf * C::TILE_BYTES;
+        for (int k = hw; k < nb; k += kThreads / 16)
+            decode_pair<FMT, BF16>(tile + k * C::BYTES, h, sgrid, p.out, t * kTileBlocks + k);
+        __syncthreads();  // the buffer is refilled next iteration
     }
+    cp_async_wait<0>();
 }
 
 template <int FMT, bool BF16>
 cudaError_t launch(const DecodeParams& p, int num_sms, cudaStream_t s) {
-    const int64_t warps_needed = (p.nblocks + kUnroll - 1) / kUnroll;
-    const int64_t ctas_needed = (warps_needed + kThreads / 32 - 1) / (kThreads / 32);
-    const int64_t cap = 8LL * num_sms;  // 8 CTAs of 256 threads fill an SM
-    const int64_t ctas = ctas_needed < cap ? ctas_needed : cap;
-    decode_kernel<FMT, BF16><<<static_cast<unsigned>(ctas), kThreads, 0, s>>>(p);
+    using C = DecodeCfg<FMT>;
+    auto kern = decode_kernel<FMT, BF16>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem);
+    if (err != cudaSuccess) return err;
+    const int64_t ntiles = (p.nblocks + kTileBlocks - 1) / kTileBlocks;
+    const int64_t cap = static_cast<int64_t>(kCtasPerSm) * num_sms;
+    const int64_t ctas = ntiles < cap ? ntiles : cap;
+    kern<<<static_cast<unsigned>(ctas), kThreads, C::smem, s>>>(p);
     return cudaGetLastError();
 }
 

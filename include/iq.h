@@ -123,7 +123,8 @@ iq_status iq_encode(const iq_desc *desc, const uint16_t *w, int64_t batch, int64
 /*
  * Decode nblocks contiguous payload blocks into [nblocks][256] values, fp32 (exact) or bf16
  * (round to nearest even of the exact value). Output is independent of how blocks are chunked.
- * payload must be 2-byte aligned and out 16-byte aligned (IQ_EINVAL otherwise).
+ * payload must be 2-byte aligned and out 32-byte aligned (IQ_EINVAL otherwise). The grid must
+ * lie in the format's alphabet (what iq_encode checks); other grid values decode unspecified.
  */
 iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks, int32_t out_dtype,
                     void *out, cudaStream_t stream);
