@@ -66,18 +66,27 @@ def alu_peak_tops(mhz: float) -> float:
     return SMS * FP32_LANES * mhz * 1e6 / 1e12
 
 
-def kernel_traffic(name: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+def kernel_traffic(name: str, workload: str, blocks: int):
+    """DRAM bytes (read + write) per launch from a committed ncu capture, if the kernel source is
+    unchanged since: the capture of this workload, else one of the same kernel scaled by the blocks
+    processed (its traffic grows in proportion). Returns (bytes or None, note)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
-    rec = json.load(open(path)).get(name)
-    if not rec:
-        return None
+        return None, "no capture"
+    table = json.load(open(path))
+    rec = table.get(f"{name}@{workload}")
+    scaled = False
+    if rec is None:
+        cands = [v for k, v in table.items() if k.startswith(name + "@") and "#" not in k]
+        if not cands:
+            return None, "no capture"
+        rec, scaled = cands[0], True
     src = os.path.join(ROOT, rec["source"])
     if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
-        return None
-    return rec["bytes_per_launch"]
+        return None, "kernel changed since the capture"
+    if scaled:
+        return int(rec["bytes_per_launch"] * blocks / rec["blocks"]), f"scaled by blocks from profiles/{rec['capture']}"
+    return rec["bytes_per_launch"], f"profiles/{rec['capture']}"
 
 
 class Clocks:
@@ -304,10 +313,10 @@ def decode_roofline(wl: Workload, dev, peaks):
     nbytes = big.shape[0] * (B + 512)
     gbs = nbytes / ms / 1e6
     del big, out, flush
+    traffic, note = kernel_traffic("decode_kernel", "iq1s_decode_1m_blocks", int(big.shape[0]))
     return {"kernel": "decode_kernel (bf16 out)", "blocks": int(flat.shape[0] * reps), "bytes_per_launch": nbytes,
             "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
-            "frac": round(gbs / peaks["hbm_gbs"], 4),
-            "traffic": kernel_traffic("decode_kernel")}
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic, "traffic_source": note}
 
 
 # ------------------------------------------------------------------------------------ oracle arm
@@ -475,17 +484,18 @@ def main():
 
     clocks = clk.summary()
     dom_avg = statistics.mean(dom_ms)
+    traffic, tnote = kernel_traffic(wl.dominant, args.workload, wl.nblocks)
     if wl.kind == "decode":
         nbytes = wl.nblocks * (iq.BLOCK_BYTES[wl.fmt] + 512)
         gbs = nbytes / (dom_avg / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": wl.dominant, "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": kernel_traffic(wl.dominant),
-                "bytes_per_launch": nbytes, "ms_per_launch": round(dom_avg, 4)}
+                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "traffic_source": tnote, "bytes_per_launch": nbytes, "ms_per_launch": round(dom_avg, 4)}
     else:
         achieved = wl.ops_per_launch / (dom_avg / 1e3) / 1e12
         peak = alu_peak_tops(peaks["sm_max_mhz"])
         roof = {"bound": "alu", "kernel": wl.dominant, "achieved": round(achieved, 3), "peak": round(peak, 3),
-                "unit": "Top/s", "frac": round(achieved / peak, 4), "traffic": kernel_traffic(wl.dominant),
+                "unit": "Top/s", "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_source": tnote,
                 "ops_per_launch": wl.ops_per_launch, "ms_per_launch": round(dom_avg, 4),
                 "peak_basis": f"{SMS} SMs x {FP32_LANES} FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (1 op/lane/clock)"}
         if clocks:
