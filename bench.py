@@ -140,6 +140,20 @@ class Clocks:
                 "samples": len(mhz)}
 
 
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The largest value any rank holds (all_reduce MAX); the value itself on a single process."""
+    if dist is None or not dist.is_initialized():
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput in M units/s: every rank processes its own units in the max time."""
+    return world * units_per_rank / (ms_per_step_max / 1e3) / 1e6
+
+
 # ------------------------------------------------------------------------------------ workloads
 
 class Workload:
@@ -447,14 +461,10 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = sum(s.elapsed_time(e) for s, e in step_ev)
+    step_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in step_ev), dist, dev)
     dom_ms = [s.elapsed_time(e) for s, e in dom_ev]
-    if dist is not None:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
     ms_per_step = step_ms / args.steps
-    value = world * wl.units / (ms_per_step / 1e3) / 1e6
+    value = weak_scaling_value(wl.units, world, ms_per_step)
 
     # end to end through the public API from pinned host memory (same stream, events)
     host, h2d, d2h = wl.host_buffers()
@@ -468,12 +478,8 @@ def main():
         wl.e2e_step(host)
     e.record()
     torch.cuda.synchronize()
-    e2e_ms = s.elapsed_time(e) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * wl.units / (e2e_ms / 1e3) / 1e6
+    e2e_ms = max_over_ranks(s.elapsed_time(e) / e2e_steps, dist, dev)
+    e2e_value = weak_scaling_value(wl.units, world, e2e_ms)
 
     dec = decode_roofline(wl, dev, peaks) if rank == 0 else None
     if dist is not None:
