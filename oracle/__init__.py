@@ -52,7 +52,7 @@ def _load(path: str | None = None):
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
         lib.orc_encode.restype = ctypes.c_uint32
-        lib.orc_encode.argtypes = [ctypes.c_int, P, ctypes.c_float, P, i64, i64, P, P, ctypes.c_int, P]
+        lib.orc_encode.argtypes = [ctypes.c_int, P, ctypes.c_float, P, i64, i64, P, P, ctypes.c_int, P, P]
         lib.orc_decode.restype = None
         lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
         lib.orc_choice_search.restype = None
@@ -120,10 +120,11 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
 
 
 def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choices=None,
-           every_choice: bool = False):
+           every_choice: bool = False, scales=None):
     """Encode a [rows, cols] bf16 weight. Returns (payload uint8, flags).
 
     payload: [rows, cols/256, B], or [16, rows, cols/256, B] with every_choice.
+    scales: optional [rows, cols/256] fp16 values (or their uint16 bits): encode under these d.
     """
     lib = _load()
     wb = _bf16_bits(w)
@@ -135,10 +136,14 @@ def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choice
     grid = np.ascontiguousarray(grid, dtype=np.int8)
     imp = None if importance is None else np.ascontiguousarray(np.asarray(importance, dtype=np.float32))
     ch = None if choices is None else np.ascontiguousarray(np.asarray(choices, dtype=np.uint8))
+    sc = None
+    if scales is not None:
+        sc = np.asarray(scales)
+        sc = np.ascontiguousarray(sc.view(np.uint16) if sc.dtype == np.float16 else sc.astype(np.uint16))
     shape = (NUM_CHOICES, rows, nblk, B) if every_choice else (rows, nblk, B)
     out = np.zeros(shape, dtype=np.uint8)
     flags = lib.orc_encode(FMT[fmt], _ptr(grid), float(anchor), _ptr(wb), rows, cols, _ptr(imp),
-                           _ptr(ch), int(bool(every_choice)), _ptr(out))
+                           _ptr(ch), int(bool(every_choice)), _ptr(sc), _ptr(out))
     return out, int(flags)
 
 
