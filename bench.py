@@ -84,7 +84,7 @@ def kernel_traffic(name: str, workload: str, blocks: int):
     src = os.path.join(ROOT, rec["source"])
     if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["sha256"]:
         return None, "kernel changed since the capture"
-    if scaled:
+    if scaled or rec["blocks"] != blocks:
         return int(rec["bytes_per_launch"] * blocks / rec["blocks"]), f"scaled by blocks from profiles/{rec['capture']}"
     return rec["bytes_per_launch"], f"profiles/{rec['capture']}"
 
@@ -324,11 +324,12 @@ def decode_roofline(wl: Workload, dev, peaks):
         torch.cuda.synchronize()
         times.append(s.elapsed_time(e))
     ms = statistics.median(times)
-    nbytes = big.shape[0] * (B + 512)
+    nblocks = int(big.shape[0])
+    nbytes = nblocks * (B + 512)
     gbs = nbytes / ms / 1e6
     del big, out, flush
-    traffic, note = kernel_traffic("decode_kernel", "iq1s_decode_1m_blocks", int(big.shape[0]))
-    return {"kernel": "decode_kernel (bf16 out)", "blocks": int(flat.shape[0] * reps), "bytes_per_launch": nbytes,
+    traffic, note = kernel_traffic("decode_kernel", "iq1s_decode_1m_blocks", nblocks)
+    return {"kernel": "decode_kernel (bf16 out)", "blocks": nblocks, "bytes_per_launch": nbytes,
             "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
             "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic, "traffic_source": note}
 

@@ -61,7 +61,7 @@ def load_library(path: str = LIB_PATH):
     lib.iq_num_choices.restype = i32
     lib.iq_num_choices.argtypes = [i32]
     lib.iq_encode.restype = ctypes.c_int
-    lib.iq_encode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, i64, i64, P, i64, P, i32, P, P, P]
+    lib.iq_encode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, i64, i64, P, i64, P, P, i64, i32, P, P, P]
     lib.iq_decode.restype = ctypes.c_int
     lib.iq_decode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i32, P, P]
     lib.iq_choice_search.restype = ctypes.c_int
@@ -110,10 +110,12 @@ def _fmt_of(desc: IQDesc) -> str:
 def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = None,
               choices: torch.Tensor | None = None, every_choice: bool = False,
               out: torch.Tensor | None = None, flags: torch.Tensor | None = None, stream=None,
-              raise_on_flags: bool = True) -> torch.Tensor:
+              raise_on_flags: bool = True, scales: torch.Tensor | None = None) -> torch.Tensor:
     """Encode bf16 weights [rows, cols] or [batch, rows, cols] (last dim contiguous).
 
     importance: fp32 [cols] or [batch, cols]; choices: uint8 [..., rows, cols/256, G].
+    scales: static block scales, either fp16 [..., rows, cols/256] (contiguous) or an existing
+    payload uint8 [..., rows, cols/256, B] whose d fields are read in place.
     Returns the payload uint8 [(16,) (batch,) rows, cols/256, B]. With raise_on_flags (default)
     the call synchronises and raises on a device-side finding; pass a flags tensor and
     raise_on_flags=False to stay asynchronous, or flags=False to skip the findings word
@@ -143,6 +145,19 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
         if choices.numel() != batch * rows * (cols // 256) * CHOICE_GROUPS[fmt] or not choices.is_contiguous():
             raise IQError(f"choices must be a contiguous uint8 tensor of {want} elements")
         ch_ptr = choices.data_ptr()
+    sc_ptr, sc_stride = None, 0
+    nb = batch * rows * (cols // 256)
+    if scales is not None:
+        if scales.device != w.device or not scales.is_contiguous():
+            raise IQError("scales must be a contiguous tensor on the weight's device")
+        if scales.dtype == torch.float16 and scales.numel() == nb:
+            sc_stride = 1
+        elif scales.dtype == torch.uint8 and scales.shape[-1] == BLOCK_BYTES[fmt] and \
+                scales.numel() == nb * BLOCK_BYTES[fmt]:
+            sc_stride = BLOCK_BYTES[fmt] // 2
+        else:
+            raise IQError(f"scales must be fp16 with {nb} elements or a payload of {nb} blocks")
+        sc_ptr = scales.data_ptr()
     shape = ((NUM_CHOICES,) if every_choice else ()) + ((batch,) if batched else ()) + \
         (rows, cols // 256, BLOCK_BYTES[fmt])
     if out is None:
@@ -153,7 +168,8 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
         flags = torch.empty(1, dtype=torch.int32, device=w.device)
     flags_ptr = None if flags is False else flags.data_ptr()
     _check(lib.iq_encode(ctypes.byref(desc), w.data_ptr(), batch, rows, cols, ldw, wbs, imp_ptr, imp_bs,
-                         ch_ptr, int(bool(every_choice)), out.data_ptr(), flags_ptr, _stream(stream)))
+                         ch_ptr, sc_ptr, sc_stride, int(bool(every_choice)), out.data_ptr(), flags_ptr,
+                         _stream(stream)))
     if raise_on_flags and flags is not False:
         raise_for_flags(flags)
     return out

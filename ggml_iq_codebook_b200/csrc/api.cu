@@ -69,8 +69,8 @@ int32_t iq_num_choices(int32_t fmt) {
 
 iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64_t rows, int64_t cols,
                     int64_t ldw, int64_t w_batch_stride, const float* importance,
-                    int64_t imp_batch_stride, const uint8_t* choices, int32_t every_choice,
-                    uint8_t* payload, uint32_t* flags, cudaStream_t stream) {
+                    int64_t imp_batch_stride, const uint8_t* choices, const uint16_t* scales,
+                    int64_t scales_stride, int32_t every_choice, uint8_t* payload, uint32_t* flags, cudaStream_t stream) {
     iq_status st = check_desc(desc);
     if (st != IQ_OK) return st;
     if (w == nullptr || payload == nullptr) return IQ_EINVAL;
@@ -83,7 +83,8 @@ iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64
     }
     if (every_choice != 0 && every_choice != 1) return IQ_EINVAL;
     if (every_choice && choices != nullptr) return IQ_EINVAL;
-    if (!aligned(payload, 2)) return IQ_EINVAL;
+    if (!aligned(payload, 2) || (scales != nullptr && (!aligned(scales, 2) || scales_stride < 1)))
+        return IQ_EINVAL;
     int sms = 0;
     if ((st = device_sms(&sms)) != IQ_OK) return st;
     if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
@@ -97,6 +98,8 @@ iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64
     p.imp = importance;
     p.imp_bstride = importance != nullptr ? imp_batch_stride : 0;
     p.choices = choices;
+    p.scales = scales;
+    p.scales_stride = scales != nullptr ? scales_stride : 0;
     p.payload = payload;
     p.flags = flags;
     p.grid = desc->grid;

@@ -134,7 +134,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
         f = __reduce_or_sync(0xffffffffu, f);
         const float amax = warp_max(am);
         uint16_t d_half = 0;
-        if (f == 0 && !bad) {
+        if (p.scales != nullptr) {
+            d_half = __ldg(p.scales + b * p.scales_stride);
+            if (given_d_bad(d_half)) f |= IQ_FLAG_RANGE;
+        } else if (f == 0 && !bad) {
             d_half = predict_d(amax, 217.0f, p.anchor);
             if ((d_half & 0x7FFFu) == 0x7C00u) f = IQ_FLAG_RANGE;
         }

@@ -14,6 +14,8 @@ struct EncodeParams {
     const float* imp;  // nullptr: all ones
     int64_t imp_bstride;
     const uint8_t* choices;  // kFixed only
+    const uint16_t* scales;  // nullptr: predict d from amax; else fp16 bits of block b's d at
+    int64_t scales_stride;   // scales[b * scales_stride]
     uint8_t* payload;
     uint32_t* flags;
     const int8_t* grid;

@@ -59,7 +59,7 @@ typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 /* device-side findings, ORed into *flags */
 #define IQ_FLAG_NONFINITE 1u  /* a weight is NaN or +-inf                                 */
 #define IQ_FLAG_IMPORTANCE 2u /* an importance value is NaN, +-inf or negative            */
-#define IQ_FLAG_RANGE 4u      /* the block scale d rounds to fp16 infinity                 */
+#define IQ_FLAG_RANGE 4u      /* d rounds to fp16 infinity, or a given d is < 0, inf or NaN */
 #define IQ_FLAG_CHOICE 8u     /* a given choice is >= 16                                  */
 #define IQ_FLAG_GRID 16u      /* a grid value lies outside the format's alphabet           */
 
@@ -100,6 +100,13 @@ int32_t iq_num_choices(int32_t fmt);
  *     values must be finite and >= 0 (PR #2723 review), else IQ_FLAG_IMPORTANCE.
  *   choices: NULL, or uint8 [batch][rows][cols/256][G] forcing each choice group's choice
  *     (PR #3157); entries and signs are still searched under it.
+ *   scales: NULL to predict each block's d from its amax, or fp16 bit patterns giving every
+ *     block's d (static scales, PR #3197, its "Static scales" item): block n of the flattened
+ *     [batch][rows][cols/256] order takes d = scales[n * scales_stride] and is searched and packed
+ *     under it whatever its amax. scales_stride >= 1 (uint16 elements): 1 for a dense array, or
+ *     B/2 to read the d of an existing payload in place (a block's d is its first two bytes).
+ *     A negative, infinite or NaN d gives the all-zero payload and IQ_FLAG_RANGE; d = +-0 gives
+ *     the all-zero payload. Works with every mode.
  *   every_choice: 0, or 1 to write all 16 choices' payloads in one sweep (PR #3159):
  *     payload c equals the encode with choices = full(c). Must be 0 when choices != NULL.
  *   payload: uint8 [batch][rows][cols/256][B], or [16][batch][rows][cols/256][B] with every_choice.
@@ -111,14 +118,15 @@ int32_t iq_num_choices(int32_t fmt);
  *          8th sign by even parity); 66..73 sixteen 4-bit local scales, sub-block 2i in the low
  *          nibble of byte 66+i.
  * Value of a weight: IQ1_S d (2 ls + 1)(q + delta); IQ2_XS d (2 ls + 1) g sign.
- * amax == 0, or d rounding to fp16 zero, gives the all-zero payload ([#2450]).
+ * Without scales, amax == 0 or d rounding to fp16 zero gives the all-zero payload ([#2450]).
  * Alignment: w and importance 16-byte aligned, ldw and w_batch_stride multiples of 8 elements,
- * imp_batch_stride a multiple of 4, payload 2-byte aligned, grid 16-byte aligned (IQ_EINVAL).
+ * imp_batch_stride a multiple of 4, payload and scales 2-byte aligned, grid 16-byte aligned
+ * (IQ_EINVAL).
  */
 iq_status iq_encode(const iq_desc *desc, const uint16_t *w, int64_t batch, int64_t rows, int64_t cols,
                     int64_t ldw, int64_t w_batch_stride, const float *importance,
-                    int64_t imp_batch_stride, const uint8_t *choices, int32_t every_choice,
-                    uint8_t *payload, uint32_t *flags, cudaStream_t stream);
+                    int64_t imp_batch_stride, const uint8_t *choices, const uint16_t *scales,
+                    int64_t scales_stride, int32_t every_choice, uint8_t *payload, uint32_t *flags, cudaStream_t stream);
 
 /*
  * Decode nblocks contiguous payload blocks into [nblocks][256] values, fp32 (exact) or bf16
