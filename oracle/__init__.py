@@ -1,7 +1,7 @@
 """CPU oracle for the GGML IQ encoder path -- TEST INFRASTRUCTURE ONLY.
 
-A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ2_XS encoder, decoder and
-local-Hessian choice search, with this thin ctypes wrapper. It is the yardstick the CUDA library is
+A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS encoder and decoder,
+and the local-Hessian choice search (IQ1_S, IQ2_XS), with this thin ctypes wrapper. It is the yardstick the CUDA library is
 checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import it; the library never does, and the two share no code.
 
@@ -22,9 +22,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "iq_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-FMT = {"iq1_s": 1, "iq2_xs": 2}
-BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74}
-CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16}
+FMT = {"iq1_s": 1, "iq2_xs": 2, "iq1_m": 3}
+BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74, "iq1_m": 56}
+CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16, "iq1_m": 16}
+CHOICES = {"iq1_s": 16, "iq2_xs": 16, "iq1_m": 8}
 NUM_CHOICES = 16
 
 FLAG_NONFINITE = 1
@@ -123,7 +124,8 @@ def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choice
            every_choice: bool = False, scales=None):
     """Encode a [rows, cols] bf16 weight. Returns (payload uint8, flags).
 
-    payload: [rows, cols/256, B], or [16, rows, cols/256, B] with every_choice.
+    payload: [rows, cols/256, B], or [C, rows, cols/256, B] with every_choice (C = 16; 8 for iq1_m).
+    anchor is ignored for iq1_m, whose anchor follows each block's peak-to-RMS.
     scales: optional [rows, cols/256] fp16 values (or their uint16 bits): encode under these d.
     """
     lib = _load()
@@ -140,7 +142,7 @@ def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choice
     if scales is not None:
         sc = np.asarray(scales)
         sc = np.ascontiguousarray(sc.view(np.uint16) if sc.dtype == np.float16 else sc.astype(np.uint16))
-    shape = (NUM_CHOICES, rows, nblk, B) if every_choice else (rows, nblk, B)
+    shape = (CHOICES[fmt], rows, nblk, B) if every_choice else (rows, nblk, B)
     out = np.zeros(shape, dtype=np.uint8)
     flags = lib.orc_encode(FMT[fmt], _ptr(grid), float(anchor), _ptr(wb), rows, cols, _ptr(imp),
                            _ptr(ch), int(bool(every_choice)), _ptr(sc), _ptr(out))
