@@ -49,7 +49,8 @@ L2_FLUSH_BYTES = 256 << 20
 #     own-block scores 16 x 16 x (256 + 16 + 15), gradient 256 x 256, two sweeps of
 #     16 groups x 16 choices x (256 + 5 x 16 - 1) gains; gradient updates after a switch are
 #     data dependent and not counted: 310,528 ops.
-OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432}
+#   IQ1_M runs IQ1_S's search (same 2048 x 16 candidates per group): 2,949,120 ops per block.
+OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120}
 CHOICE_OPS_PER_ROW_BLOCK = 310_528
 SMS, FP32_LANES = 148, 128
 
@@ -163,11 +164,16 @@ class Workload:
         self.name, self.dev, self.peaks = name, dev, peaks
         g1 = torch.from_numpy(synth.iq1s_grid()).to(dev)
         g2 = torch.from_numpy(synth.iq2xs_grid()).to(dev)
-        self.desc = {"iq1_s": iq.make_desc("iq1_s", g1), "iq2_xs": iq.make_desc("iq2_xs", g2)}
+        self.desc = {"iq1_s": iq.make_desc("iq1_s", g1), "iq2_xs": iq.make_desc("iq2_xs", g2),
+                     "iq1_m": iq.make_desc("iq1_m", g1)}
         self.launches_per_step = 2
         if name == "iq1s_4096x4096_weighted":
             wl = synth.workload_iq1s_4096x4096_weighted()
             self._encode_decode(wl, "IQ1_S importance-weighted encode + bf16 decode, 4096x4096 bf16 "
+                                    "N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))")
+        elif name == "iq1m_4096x4096_weighted":
+            wl = dict(synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m")
+            self._encode_decode(wl, "IQ1_M importance-weighted encode + bf16 decode, 4096x4096 bf16 "
                                     "N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))")
         elif name == "iq2xs_8192x4096":
             wl = synth.workload_iq2xs_8192x4096()
@@ -210,7 +216,7 @@ class Workload:
         self.units = self.w.numel()
         self.nblocks = self.units // 256
         self.text = text
-        self.dominant = f"{self.fmt.replace('_', '')}_encode_kernel"
+        self.dominant = "iq2xs_encode_kernel" if self.fmt == "iq2_xs" else "iq1_encode_kernel"
         self.ops_per_launch = self.nblocks * OPS_PER_BLOCK[self.fmt]
         # validate once (findings word + raise) before anything is timed
         iq.iq_encode(self.desc[self.fmt], self.w, self.imp, out=self.payload)
@@ -328,7 +334,10 @@ def decode_roofline(wl: Workload, dev, peaks):
     nbytes = nblocks * (B + 512)
     gbs = nbytes / ms / 1e6
     del big, out, flush
-    traffic, note = kernel_traffic("decode_kernel", "iq1s_decode_1m_blocks", nblocks)
+    if wl.fmt == "iq1_s":
+        traffic, note = kernel_traffic("decode_kernel", "iq1s_decode_1m_blocks", nblocks)
+    else:
+        traffic, note = None, f"no capture of the {wl.fmt} decode"
     return {"kernel": "decode_kernel (bf16 out)", "blocks": nblocks, "bytes_per_launch": nbytes,
             "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
             "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic, "traffic_source": note}
@@ -355,11 +364,12 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
             fmt = "iq1_s"
         else:
             wl = {"iq1s_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
+                  "iq1m_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
                   "iq1s_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
                   "iq2xs_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq1s_64x256": synth.workload_iq1s_64x256}[name]()
-            w, imp, fmt = wl["w"], wl["importance"], wl["fmt"]
-        g = synth.iq1s_grid() if fmt == "iq1_s" else synth.iq2xs_grid()
+            w, imp, fmt = wl["w"], wl["importance"], ("iq1_m" if name.startswith("iq1m") else wl["fmt"])
+        g = synth.iq2xs_grid() if fmt == "iq2_xs" else synth.iq1s_grid()
 
         def run(r):
             p, _ = oracle.encode(fmt, g, iq.DEFAULT_ANCHOR[fmt], w[:r], importance=imp)

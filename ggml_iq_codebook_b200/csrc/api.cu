@@ -37,7 +37,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 iq_status check_desc(const iq_desc* d) {
     if (d == nullptr || d->grid == nullptr) return IQ_EINVAL;
-    if (d->fmt == IQ_FMT_IQ1_S) {
+    if (d->fmt == IQ_FMT_IQ1_S || d->fmt == IQ_FMT_IQ1_M) {
         if (d->grid_entries != 2048) return IQ_EINVAL;
     } else if (d->fmt == IQ_FMT_IQ2_XS) {
         if (d->grid_entries != 512) return IQ_EINVAL;
@@ -45,7 +45,8 @@ iq_status check_desc(const iq_desc* d) {
         return IQ_EINVAL;
     }
     if (!aligned(d->grid, 16)) return IQ_EINVAL;
-    if (!std::isfinite(d->anchor) || !(d->anchor > 0.0f)) return IQ_EINVAL;
+    // IQ1_M derives its anchor from each block; the others take it from the descriptor.
+    if (d->fmt != IQ_FMT_IQ1_M && (!std::isfinite(d->anchor) || !(d->anchor > 0.0f))) return IQ_EINVAL;
     return IQ_OK;
 }
 
@@ -56,15 +57,15 @@ iq_status launched(cudaError_t e) { return e == cudaSuccess ? IQ_OK : IQ_ECUDA; 
 extern "C" {
 
 size_t iq_block_bytes(int32_t fmt) {
-    return fmt == IQ_FMT_IQ1_S ? 50 : fmt == IQ_FMT_IQ2_XS ? 74 : 0;
+    return fmt == IQ_FMT_IQ1_S ? 50 : fmt == IQ_FMT_IQ2_XS ? 74 : fmt == IQ_FMT_IQ1_M ? 56 : 0;
 }
 
 int32_t iq_choice_groups(int32_t fmt) {
-    return fmt == IQ_FMT_IQ1_S ? 8 : fmt == IQ_FMT_IQ2_XS ? 16 : 0;
+    return fmt == IQ_FMT_IQ1_S ? 8 : (fmt == IQ_FMT_IQ2_XS || fmt == IQ_FMT_IQ1_M) ? 16 : 0;
 }
 
 int32_t iq_num_choices(int32_t fmt) {
-    return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS) ? 16 : 0;
+    return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS) ? 16 : fmt == IQ_FMT_IQ1_M ? 8 : 0;
 }
 
 iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64_t rows, int64_t cols,
@@ -106,8 +107,8 @@ iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64
     p.anchor = desc->anchor;
     p.nb = batch * rows * (cols / 256);
     const int mode = every_choice ? iqk::kEvery : (choices != nullptr ? iqk::kFixed : iqk::kSearch);
-    return launched(desc->fmt == IQ_FMT_IQ1_S ? iqk::launch_iq1s_encode(p, mode, sms, stream)
-                                              : iqk::launch_iq2xs_encode(p, mode, sms, stream));
+    return launched(desc->fmt == IQ_FMT_IQ2_XS ? iqk::launch_iq2xs_encode(p, mode, sms, stream)
+                                               : iqk::launch_iq1_encode(desc->fmt, p, mode, sms, stream));
 }
 
 iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks, int32_t out_dtype,
@@ -134,6 +135,7 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
                            int64_t payload_ld, uint32_t* flags, cudaStream_t stream) {
     iq_status st = check_desc(desc);
     if (st != IQ_OK) return st;
+    if (desc->fmt == IQ_FMT_IQ1_M) return IQ_EUNSUPPORTED;
     if (w == nullptr || hess == nullptr || cand == nullptr || picks == nullptr || payload == nullptr)
         return IQ_EINVAL;
     if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;
@@ -174,7 +176,7 @@ const char* iq_status_string(iq_status s) {
         case IQ_EINVAL: return "invalid argument";
         case IQ_ESHAPE: return "invalid shape (empty, or columns not a multiple of 256)";
         case IQ_ECUDA: return "CUDA error";
-        case IQ_EUNSUPPORTED: return "device is not sm_100";
+        case IQ_EUNSUPPORTED: return "device is not sm_100, or the call does not take this format";
         default: return "unknown status";
     }
 }

@@ -1,4 +1,5 @@
-// iq1s_encode.cu -- IQ1_S encoder: weighted exhaustive shifted-grid search + pack (sm_100a).
+// iq1_encode.cu -- IQ1_S and IQ1_M encoders: weighted exhaustive shifted-grid search + pack
+// (sm_100a).
 //
 // Method (PR #2723 "Weight the IQ1 encoders by the square root of GPTQ's Hessian diagonal";
 // PR #2450 review comments): each 8-weight group x is approximated by s (q + delta) with q one
@@ -14,6 +15,12 @@
 //   per choice A_d = fma(d^2, W, fma(2 d, R, A));  C_d = fma(d, Tall, C);  m = fma(s, A_d, C_d)
 //   per (group, c)     argmin_q m (lowest q on ties), e = s * m_min
 //   per (sub-block, c) E = (e0 + e1) + (e2 + e3);  choice = argmin_c E (lowest c on ties)
+//
+// IQ1_M (PR #2513 codec, PR #2595 CUDA encoder commit texts) runs the same search and selects
+// differently: a choice group is two 8-weight groups sharing ls (8 choices); per group and ls the
+// delta with the smaller m wins (+1/8 on equal m), e = s * m, E = e_even + e_odd, lowest ls on
+// ties. Its d anchor is clamp(0.58 + 0.035 amax / rms, 0.65, 0.95), with rms = sqrt(ss / 256):
+// each lane sums its 8 squares in order, the 32 lane sums meet in the xor-butterfly tree.
 //
 // Kernel design (B200): one warp per 256-weight block, one lane per group, so the 2048-entry
 // loop is warp-uniform: the entry's four subset-sum row offsets come from one broadcast
@@ -33,6 +40,15 @@ constexpr int kWarps = 8;                      // warps per CTA
 constexpr int kGridBytes = kIq1sEntries * 16;  // uint4 of 4 table-row byte offsets per entry
 constexpr int kTabBytes = 32 * 32 * 8;         // 32 rows x 32 lanes x float2, per warp
 constexpr int kSmemBytes = kGridBytes + kWarps * kTabBytes;
+
+template <int FMT>
+struct Iq1Cfg {
+    static constexpr bool M = FMT == IQ_FMT_IQ1_M;
+    static constexpr int BYTES = M ? kIq1mBytes : kIq1sBytes;
+    static constexpr int NCH = M ? kIq1mChoices : kChoices;  // choices per choice group
+    static constexpr int G = M ? 16 : 8;                     // choice groups per block
+    static constexpr int LANES_PER_CHOICE = 32 / G;          // groups (lanes) per choice group
+};
 
 struct Terms {
     float Ap, An, Cp, Cn;  // A_delta and C_delta for delta = +1/8 and -1/8
@@ -56,8 +72,9 @@ __device__ __forceinline__ Terms entry_terms(const char* smem, uint32_t lane_bas
     return t;
 }
 
+template <int BYTES>
 __device__ __forceinline__ void write_zero_block(uint8_t* out, int lane) {
-    for (int i = lane; i < kIq1sBytes / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
+    for (int i = lane; i < BYTES / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
 }
 
 // Pack one block: lane = group, idx = its entry, c = its sub-block's choice.
@@ -71,8 +88,28 @@ __device__ __forceinline__ void pack_block(uint8_t* out, int lane, int idx, int 
     if (lane == 0) *reinterpret_cast<uint16_t*>(out) = d_half;
 }
 
-template <int MODE, int K>
-__global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const EncodeParams p) {
+// Pack one IQ1_M block: lane = group, idx = its entry, neg = its delta bit, ls = its choice
+// group's local scale. Bytes 0..31 low index bytes; 32..47 a nibble per group (even group low);
+// 48..55 four scale words: ls of choice groups 4i..4i+3 at shifts 0,3,6,9, d's nibble i on top.
+__device__ __forceinline__ void pack_block_m(uint8_t* out, int lane, int idx, int ls, int neg, uint16_t d_half) {
+    out[lane] = static_cast<uint8_t>(idx & 0xFF);
+    uint32_t v = (static_cast<uint32_t>((idx >> 8) & 7) | (static_cast<uint32_t>(neg) << 3)) << (4 * (lane & 1));
+    v |= __shfl_xor_sync(0xffffffffu, v, 1);
+    if ((lane & 1) == 0) out[32 + (lane >> 1)] = static_cast<uint8_t>(v);
+    uint32_t wv = (lane & 1) ? 0u : static_cast<uint32_t>(ls) << (3 * ((lane >> 1) & 3));
+    wv |= __shfl_xor_sync(0xffffffffu, wv, 1);
+    wv |= __shfl_xor_sync(0xffffffffu, wv, 2);
+    wv |= __shfl_xor_sync(0xffffffffu, wv, 4);
+    if ((lane & 7) == 0) {
+        const int i = lane >> 3;
+        *reinterpret_cast<uint16_t*>(out + 48 + 2 * i) =
+            static_cast<uint16_t>(wv | ((static_cast<uint32_t>(d_half >> (4 * i)) & 15u) << 12));
+    }
+}
+
+template <int FMT, int MODE, int K>
+__global__ void __launch_bounds__(kWarps * 32, 2) iq1_encode_kernel(const EncodeParams p) {
+    using Cfg = Iq1Cfg<FMT>;
     extern __shared__ __align__(16) char smem[];
     uint4* sgrid = reinterpret_cast<uint4*>(smem);
 
@@ -103,8 +140,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
     for (int64_t b = static_cast<int64_t>(blockIdx.x) * kWarps + warp; b < p.nb; b += stride) {
         const int64_t e = b / per_batch, rem = b - e * per_batch;
         const int64_t r = rem / p.nblk, blk = rem - r * p.nblk;
-        uint8_t* out = p.payload + b * kIq1sBytes;
-        const int64_t every_stride = p.nb * kIq1sBytes;
+        uint8_t* out = p.payload + b * Cfg::BYTES;
+        const int64_t every_stride = p.nb * Cfg::BYTES;
 
         // ---- load + validate (8 weights and importances per lane, 16-byte vector loads)
         float x[8], w[8];
@@ -127,8 +164,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
         }
         int fixed_c = 0;
         if (MODE == kFixed) {
-            fixed_c = p.choices[b * 8 + (lane >> 2)];
-            if (fixed_c >= kChoices) f |= IQ_FLAG_CHOICE;
+            fixed_c = p.choices[b * Cfg::G + lane / Cfg::LANES_PER_CHOICE];
+            if (fixed_c >= Cfg::NCH) f |= IQ_FLAG_CHOICE;
         }
         f = __reduce_or_sync(0xffffffffu, f);
         const float amax = warp_max(am);
@@ -137,14 +174,25 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
             d_half = __ldg(p.scales + b * p.scales_stride);
             if (given_d_bad(d_half)) f |= IQ_FLAG_RANGE;
         } else if (f == 0 && !bad) {
-            d_half = predict_d(amax, 16.875f, p.anchor);
+            float anchor = p.anchor;
+            if (Cfg::M) {
+                float ss = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ss = __fadd_rn(ss, __fmul_rn(x[j], x[j]));
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+                const float rms = __fsqrt_rn(__fdiv_rn(ss, 256.0f));
+                const float ratio = __fdiv_rn(amax, rms);
+                anchor = fminf(fmaxf(__fadd_rn(0.58f, __fmul_rn(0.035f, ratio)), 0.65f), 0.95f);
+            }
+            d_half = predict_d(amax, 16.875f, anchor);
             if ((d_half & 0x7FFFu) == 0x7C00u) f = IQ_FLAG_RANGE;
         }
         if (f != 0 || bad || (d_half & 0x7FFFu) == 0) {
             if (MODE == kEvery) {
-                for (int c = 0; c < kChoices; ++c) write_zero_block(out + c * every_stride, lane);
+                for (int c = 0; c < Cfg::NCH; ++c) write_zero_block<Cfg::BYTES>(out + c * every_stride, lane);
             } else {
-                write_zero_block(out, lane);
+                write_zero_block<Cfg::BYTES>(out, lane);
             }
             if (lane == 0) raise_flags(p.flags, f);
             continue;
@@ -178,6 +226,25 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
 #pragma unroll
         for (int ls = 0; ls < 8; ++ls) s[ls] = __fmul_rn(d, static_cast<float>(2 * ls + 1));
 
+        if (MODE == kFixed && Cfg::M) {
+            // The lane's local scale is given; both deltas are searched, each keeping its lowest
+            // entry, and the negative shift wins only with a strictly smaller m.
+            float sv = s[0];
+#pragma unroll
+            for (int ls = 1; ls < 8; ++ls) if (fixed_c == ls) sv = s[ls];
+            float bp = INFINITY, bn = INFINITY;
+            int qp = 0, qn = 0;
+#pragma unroll 4
+            for (int q = 0; q < kIq1sEntries; ++q) {
+                const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+                const float mp = __fmaf_rn(sv, tm.Ap, tm.Cp), mn = __fmaf_rn(sv, tm.An, tm.Cn);
+                if (mp < bp) { bp = mp; qp = q; }
+                if (mn < bn) { bn = mn; qn = q; }
+            }
+            const int neg = bn < bp;
+            pack_block_m(out, lane, neg ? qn : qp, fixed_c, neg, d_half);
+            continue;
+        }
         if (MODE == kFixed) {
             // One choice per lane: direct argmin with the index (lowest entry on ties).
             float sv = s[0];
@@ -247,6 +314,32 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
             return ch * K;  // not reached: the same arithmetic reproduces target
         };
 
+        if (Cfg::M) {
+            // per ls: the group's delta (bit ls of negmask: -1/8 only with a strictly smaller m)
+            uint32_t negmask = 0;
+#pragma unroll
+            for (int ls = 0; ls < kIq1mChoices; ++ls) negmask |= static_cast<uint32_t>(best[8 + ls] < best[ls]) << ls;
+            if (MODE == kEvery) {
+                for (int ls = 0; ls < kIq1mChoices; ++ls) {
+                    const int neg = (negmask >> ls) & 1;
+                    pack_block_m(out + ls * every_stride, lane, entry_of(ls + 8 * neg), ls, neg, d_half);
+                }
+                continue;
+            }
+            // e = s m under the group's delta, E = e_even + e_odd over the choice group
+            int lstar = 0;
+            float bestE = INFINITY;
+#pragma unroll
+            for (int ls = 0; ls < kIq1mChoices; ++ls) {
+                const float mm = ((negmask >> ls) & 1) ? best[8 + ls] : best[ls];
+                const float e = __fmul_rn(s[ls], mm);
+                const float E = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 1));
+                if (E < bestE) { bestE = E; lstar = ls; }
+            }
+            const int neg = (negmask >> lstar) & 1;
+            pack_block_m(out, lane, entry_of(lstar + 8 * neg), lstar, neg, d_half);
+            continue;
+        }
         if (MODE == kEvery) {
             for (int c = 0; c < kChoices; ++c) pack_block(out + c * every_stride, lane, entry_of(c), c, d_half);
             continue;
@@ -266,9 +359,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1s_encode_kernel(const Encod
     }
 }
 
-template <int MODE, int K>
+template <int FMT, int MODE, int K>
 cudaError_t launch_mode(const EncodeParams& p, int num_sms, cudaStream_t s) {
-    auto kern = iq1s_encode_kernel<MODE, K>;
+    auto kern = iq1_encode_kernel<FMT, MODE, K>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
     const int64_t ctas_needed = (p.nb + kWarps - 1) / kWarps;
@@ -279,13 +372,19 @@ cudaError_t launch_mode(const EncodeParams& p, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_iq1s_encode(const EncodeParams& p, int mode, int num_sms, cudaStream_t s) {
-    if (p.nb == 0) return cudaSuccess;
+template <int FMT>
+cudaError_t launch_fmt(const EncodeParams& p, int mode, int num_sms, cudaStream_t s) {
     switch (mode) {
-        case kSearch: return launch_mode<kSearch, 32>(p, num_sms, s);
-        case kFixed: return launch_mode<kFixed, 32>(p, num_sms, s);
-        default: return launch_mode<kEvery, 8>(p, num_sms, s);
+        case kSearch: return launch_mode<FMT, kSearch, 32>(p, num_sms, s);
+        case kFixed: return launch_mode<FMT, kFixed, 32>(p, num_sms, s);
+        default: return launch_mode<FMT, kEvery, 8>(p, num_sms, s);
     }
+}
+
+cudaError_t launch_iq1_encode(int fmt, const EncodeParams& p, int mode, int num_sms, cudaStream_t s) {
+    if (p.nb == 0) return cudaSuccess;
+    return fmt == IQ_FMT_IQ1_M ? launch_fmt<IQ_FMT_IQ1_M>(p, mode, num_sms, s)
+                               : launch_fmt<IQ_FMT_IQ1_S>(p, mode, num_sms, s);
 }
 
 }  // namespace iqk

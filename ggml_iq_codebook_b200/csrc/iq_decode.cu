@@ -1,10 +1,13 @@
-// iq_decode.cu -- IQ1_S / IQ2_XS decoders (sm_100a), HBM-bound.
+// iq_decode.cu -- IQ1_S / IQ2_XS / IQ1_M decoders (sm_100a), HBM-bound.
 //
 // Values (PR #2450 review comments):
 //   IQ1_S  x = d (2 ls + 1) (q_j + delta), index = low | ((qh >> 3i) & 7) << 8, ls = qh bits
 //          12..14, delta = -1/8 if qh bit 15 else +1/8.
 //   IQ2_XS x = d (2 ls + 1) g_j (-1)^sign_j, code = index | sign7 << 9, sign_7 = parity(sign7),
 //          ls of sub-block k in nibble (k & 1) of byte 66 + k/2.
+//   IQ1_M  (PR #2513) x = d (2 ls + 1) (q_j + delta), d = the top nibbles of the four scale words
+//          at bytes 48..55, ls of choice group k = bits 3(k%4).. of word k/4, group g's index
+//          = byte g | (nibble g of bytes 32.. & 7) << 8, delta = -1/8 if that nibble's bit 3.
 // Every value is a product of at most 20 significant bits, so the fp32 result is exact; the bf16
 // output is its round-to-nearest-even. Each block decodes independently, so the output does not
 // depend on how a caller chunks the blocks.
@@ -78,7 +81,7 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // A half-warp decodes one block from its staged payload bytes `pb` (2-byte aligned); lane
-// h = lane & 15 decodes groups 2h and 2h + 1. No int-to-float conversion on the way: a lane
+// h = lane & 15 decodes groups 2h and 2h + 1 (for IQ1_M: exactly choice group h). No int-to-float conversion on the way: a lane
 // forms the few products a group can take (IQ1_S: s (q + delta) for q in {-1, 0, 1}; IQ2_XS:
 // s g for g in {1, 3, 5, 7}), each rounded exactly as the direct formula rounds it, and picks
 // per element from the staged grid codes.
@@ -86,6 +89,28 @@ template <int FMT, bool BF16>
 __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint16_t* sgrid, void* out, int64_t b) {
     const uint16_t* pw = reinterpret_cast<const uint16_t*>(pb);
     float v[16];
+    if (FMT == IQ_FMT_IQ1_M) {
+        const uint32_t w0 = pw[24], w1 = pw[25], w2 = pw[26], w3 = pw[27];
+        const float d = half_bits_to_f32(iq1m_d_bits(w0, w1, w2, w3));
+        const uint32_t wk = pw[24 + (h >> 2)];
+        const float s = __fmul_rn(d, static_cast<float>(2 * static_cast<int>((wk >> (3 * (h & 3))) & 7u) + 1));
+        const uint32_t lw = pw[h];      // low index bytes of groups 2h, 2h + 1
+        const uint32_t nb = pb[32 + h];  // their nibbles
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t nib = (nb >> (4 * t)) & 15u;
+            const float delta = (nib & 8u) ? -0.125f : 0.125f;
+            const float vp = __fmul_rn(s, __fadd_rn(1.0f, delta));
+            const float v0 = __fmul_rn(s, __fadd_rn(0.0f, delta));
+            const float vn = __fmul_rn(s, __fadd_rn(-1.0f, delta));
+            const int idx = static_cast<int>(((lw >> (8 * t)) & 0xFFu) | ((nib & 7u) << 8));
+            const uint32_t m = sgrid[idx];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[8 * t + j] = ((m >> j) & 1u) ? vp : (((m >> (8 + j)) & 1u) ? vn : v0);
+        }
+        store16<BF16>(out, b * 32 + 2 * h, v);
+        return;
+    }
     const float d = half_bits_to_f32(pw[0]);
     if (FMT == IQ_FMT_IQ1_S) {
         const uint32_t lw = pw[1 + h];          // low index bytes of groups 2h, 2h + 1
@@ -128,14 +153,14 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
 
 template <int FMT>
 struct DecodeCfg {
-    static constexpr int BYTES = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : kIq2xsBytes;
-    static constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : kIq2xsEntries;
+    static constexpr int BYTES = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : FMT == IQ_FMT_IQ1_M ? kIq1mBytes : kIq2xsBytes;
+    static constexpr int E = FMT == IQ_FMT_IQ2_XS ? kIq2xsEntries : kIq1sEntries;
     static constexpr int TILE_BYTES = kTileBlocks * BYTES;  // a multiple of 16
     static constexpr int GRID_BYTES = (E * 2 + 15) / 16 * 16;
     static constexpr int smem = GRID_BYTES + 2 * TILE_BYTES;
 };
 
-// The grid as 16-bit codes: IQ1_S (+1 mask) | (-1 mask) << 8; IQ2_XS two bits (g - 1) / 2 per
+// The grid as 16-bit codes: IQ1_S, IQ1_M (+1 mask) | (-1 mask) << 8; IQ2_XS two bits (g - 1) / 2 per
 // element. Values outside the format's alphabet are not representable here.
 template <int FMT>
 __device__ __forceinline__ uint16_t grid_code(int2 raw) {
@@ -143,7 +168,7 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
-        if (FMT == IQ_FMT_IQ1_S) c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
+        if (FMT != IQ_FMT_IQ2_XS) c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
         else c |= (static_cast<uint32_t>((v - 1) >> 1) & 3u) << (2 * j);
     }
     return static_cast<uint16_t>(c);
@@ -211,6 +236,7 @@ cudaError_t launch(const DecodeParams& p, int num_sms, cudaStream_t s) {
 cudaError_t launch_decode(int fmt, bool bf16, const DecodeParams& p, int num_sms, cudaStream_t s) {
     if (p.nblocks == 0) return cudaSuccess;
     if (fmt == IQ_FMT_IQ1_S) return bf16 ? launch<IQ_FMT_IQ1_S, true>(p, num_sms, s) : launch<IQ_FMT_IQ1_S, false>(p, num_sms, s);
+    if (fmt == IQ_FMT_IQ1_M) return bf16 ? launch<IQ_FMT_IQ1_M, true>(p, num_sms, s) : launch<IQ_FMT_IQ1_M, false>(p, num_sms, s);
     return bf16 ? launch<IQ_FMT_IQ2_XS, true>(p, num_sms, s) : launch<IQ_FMT_IQ2_XS, false>(p, num_sms, s);
 }
 

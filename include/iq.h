@@ -12,7 +12,9 @@
  *     on equal error, even sign parity); the IQ2_S codec commit text on the PR #2525 page
  *     (IQ2_XS fixes parity by flipping the weakest element).
  *   - fixed per-group choices (PR #3157) and the one-pass every-choice encode (PR #3159);
- *   - decoding of both layouts;
+ *   - IQ1_M (PR #2513 codec and PR #2595 encoder commit texts): the IQ1_S search with a local
+ *     scale per 16 weights, a delta per 8-weight group and d kept in four scale words;
+ *   - decoding of the three layouts;
  *   - the local-Hessian choice search (PR #3158, fused in PR #3218 "[4/4] Run the local-Hessian
  *     choice search as one CUDA kernel").
  *
@@ -49,10 +51,10 @@ typedef enum {
     IQ_EINVAL = 1,        /* NULL pointer, unknown format, bad descriptor or stride          */
     IQ_ESHAPE = 2,        /* empty tensor, or cols not a multiple of 256 ([512, 384] case)     */
     IQ_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed                       */
-    IQ_EUNSUPPORTED = 4   /* the current device is not sm_100                                  */
+    IQ_EUNSUPPORTED = 4   /* the current device is not sm_100, or the call does not take the format */
 } iq_status;
 
-typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2 } iq_format;
+typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3 } iq_format;
 
 typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 
@@ -65,15 +67,18 @@ typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 
 /*
  * Codebook/convention descriptor (host struct; the grid it points to lives on the device).
- *   fmt           IQ_FMT_IQ1_S or IQ_FMT_IQ2_XS
- *   grid_entries  2048 (IQ1_S) or 512 (IQ2_XS)
- *   grid          device int8 [grid_entries][8]; IQ1_S values in {-1,0,1} (a ternary grid,
- *                 PR #2723), IQ2_XS magnitudes in {1,3,5,7}. Row q, column j multiplies weight j
- *                 of a group.
+ *   fmt           IQ_FMT_IQ1_S, IQ_FMT_IQ2_XS or IQ_FMT_IQ1_M
+ *   grid_entries  2048 (IQ1_S, IQ1_M) or 512 (IQ2_XS)
+ *   grid          device int8 [grid_entries][8]; IQ1_S and IQ1_M values in {-1,0,1} (a ternary
+ *                 grid, PR #2723; IQ1_M shares IQ1_S's, PR #2513), IQ2_XS magnitudes in {1,3,5,7}.
+ *                 Row q, column j multiplies weight j of a group.
  *   anchor        the scale predictor's anchor: d = fp16(fp32(amax / qmax) * anchor), with
  *                 qmax = 16.875 (IQ1_S, = 15 * 1.125, the largest |s (q + delta)| in units of d)
  *                 and 217 (IQ2_XS, = 31 * 7). IQ1_S uses 0.61 (PR #2450 review). The pages give
- *                 no IQ2_XS constant; this library's default is 0.9.
+ *                 no IQ2_XS constant; this library's default is 0.9. IQ1_M ignores it: its anchor
+ *                 is clamp(0.58 + 0.035 * amax / rms, 0.65, 0.95) per block (PR #2513), rms over
+ *                 the block's 256 weights (squares summed per 8-weight group in order, the 32
+ *                 group sums by a pairwise tree), with qmax = 16.875.
  */
 typedef struct {
     int32_t fmt;
@@ -82,14 +87,16 @@ typedef struct {
     float anchor;
 } iq_desc;
 
-/* Bytes per 256-weight block: 50 (IQ1_S), 74 (IQ2_XS); 0 for an unknown format. */
+/* Bytes per 256-weight block: 50 (IQ1_S), 74 (IQ2_XS), 56 (IQ1_M); 0 for an unknown format. */
 size_t iq_block_bytes(int32_t fmt);
 
 /* Choice groups per block: 8 (IQ1_S, one per 32 weights: local scale + delta sign),
- * 16 (IQ2_XS, one 4-bit local scale per 16 weights); 0 for an unknown format. */
+ * 16 (IQ2_XS, one 4-bit local scale per 16 weights; IQ1_M, one 3-bit local scale per 16 weights,
+ * each 8-weight group taking its own delta); 0 for an unknown format. */
 int32_t iq_choice_groups(int32_t fmt);
 
-/* Choices per group: 16 for both formats (IQ1_S: c = ls + 8 * [delta < 0]; IQ2_XS: c = ls). */
+/* Choices per group: 16 for IQ1_S (c = ls + 8 * [delta < 0]) and IQ2_XS (c = ls); 8 for IQ1_M
+ * (c = ls); 0 for an unknown format. */
 int32_t iq_num_choices(int32_t fmt);
 
 /*
@@ -99,17 +106,18 @@ int32_t iq_num_choices(int32_t fmt);
  *     importance[e * imp_batch_stride + col]     (imp_batch_stride 0 shares one vector)
  *     values must be finite and >= 0 (PR #2723 review), else IQ_FLAG_IMPORTANCE.
  *   choices: NULL, or uint8 [batch][rows][cols/256][G] forcing each choice group's choice
- *     (PR #3157); entries and signs are still searched under it.
+ *     (PR #3157); entries, signs and IQ1_M's per-group deltas are still searched under it.
  *   scales: NULL to predict each block's d from its amax, or fp16 bit patterns giving every
  *     block's d (static scales, PR #3197, its "Static scales" item): block n of the flattened
  *     [batch][rows][cols/256] order takes d = scales[n * scales_stride] and is searched and packed
  *     under it whatever its amax. scales_stride >= 1 (uint16 elements): 1 for a dense array, or
- *     B/2 to read the d of an existing payload in place (a block's d is its first two bytes).
+ *     B/2 to read the d of an existing IQ1_S or IQ2_XS payload in place (its first two bytes).
  *     A negative, infinite or NaN d gives the all-zero payload and IQ_FLAG_RANGE; d = +-0 gives
  *     the all-zero payload. Works with every mode.
- *   every_choice: 0, or 1 to write all 16 choices' payloads in one sweep (PR #3159):
+ *   every_choice: 0, or 1 to write all C choices' payloads in one sweep (PR #3159):
  *     payload c equals the encode with choices = full(c). Must be 0 when choices != NULL.
- *   payload: uint8 [batch][rows][cols/256][B], or [16][batch][rows][cols/256][B] with every_choice.
+ *   payload: uint8 [batch][rows][cols/256][B], or [C][batch][rows][cols/256][B] with every_choice
+ *     (C = iq_num_choices(fmt)).
  * Per block ([#2450] layouts):
  *   IQ1_S  bytes 0-1 fp16 d; 2..33 low 8 bits of the 32 group indices; 34..49 eight LE uint16 qh,
  *          one per 32-weight sub-block: bits 0..11 the high 3 index bits of its 4 groups (shifts
@@ -117,7 +125,14 @@ int32_t iq_num_choices(int32_t fmt);
  *   IQ2_XS bytes 0-1 fp16 d; 2..65 32 LE uint16 codes (9-bit index | 7-bit sign mask << 9, the
  *          8th sign by even parity); 66..73 sixteen 4-bit local scales, sub-block 2i in the low
  *          nibble of byte 66+i.
- * Value of a weight: IQ1_S d (2 ls + 1)(q + delta); IQ2_XS d (2 ls + 1) g sign.
+ *   IQ1_M  bytes 0..31 low 8 bits of the 32 group indices; 32..47 a nibble per group (group 2i in
+ *          the low nibble of byte 32+i): 3 high index bits, bit 3 set for delta = -1/8; 48..55
+ *          four LE uint16 scale words: word i holds the 3-bit ls of choice groups 4i..4i+3 at
+ *          shifts 0,3,6,9 and bits 12..15 of word i are bits 4i..4i+3 of fp16 d (PR #2513).
+ * Value of a weight: IQ1_S, IQ1_M d (2 ls + 1)(q + delta); IQ2_XS d (2 ls + 1) g sign.
+ * IQ1_M picks, per group and ls, the (delta, entry) of least error, the lower shift (+1/8) and
+ * then the lower entry on equal error (PR #2595); a choice group's error is the sum of its two
+ * groups'.
  * Without scales, amax == 0 or d rounding to fp16 zero gives the all-zero payload ([#2450]).
  * Alignment: w and importance 16-byte aligned, ldw and w_batch_stride multiples of 8 elements,
  * imp_batch_stride a multiple of 4, payload and scales 2-byte aligned, grid 16-byte aligned
@@ -139,7 +154,7 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
 
 /*
  * Local-Hessian choice search (PR #3158 steps; one fused launch as in PR #3218) for the first
- * nblk 256-column blocks of a [rows, ldw] bf16 weight.
+ * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S and IQ2_XS (IQ1_M: IQ_EUNSUPPORTED).
  *   hess: fp32 [nblk][256][256], the symmetric diagonal block of the input Hessian per block,
  *     read as H[k][i] (row k, column i) for (H v)_i.
  *   cand: the every-choice payloads of those blocks; candidate c of (row r, block b) starts at

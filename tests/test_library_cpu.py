@@ -37,9 +37,15 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_format_tables(lib):
-    assert lib.iq_block_bytes(1) == 50 and lib.iq_block_bytes(2) == 74 and lib.iq_block_bytes(3) == 0
-    assert lib.iq_choice_groups(1) == 8 and lib.iq_choice_groups(2) == 16
-    assert lib.iq_num_choices(1) == 16 and lib.iq_num_choices(2) == 16 and lib.iq_num_choices(0) == 0
+    assert lib.iq_block_bytes(1) == 50 and lib.iq_block_bytes(2) == 74 and lib.iq_block_bytes(3) == 56
+    assert lib.iq_block_bytes(4) == 0
+    assert lib.iq_choice_groups(1) == 8 and lib.iq_choice_groups(2) == 16 and lib.iq_choice_groups(3) == 16
+    assert lib.iq_num_choices(1) == 16 and lib.iq_num_choices(2) == 16 and lib.iq_num_choices(3) == 8
+    assert lib.iq_num_choices(0) == 0
+    for fmt, code in iq.IQ_FMT.items():
+        assert lib.iq_block_bytes(code) == iq.BLOCK_BYTES[fmt]
+        assert lib.iq_choice_groups(code) == iq.CHOICE_GROUPS[fmt]
+        assert lib.iq_num_choices(code) == iq.CHOICES[fmt]
     assert b"sm_100a" in lib.iq_build_info()
     assert lib.iq_status_string(2).startswith(b"invalid shape")
 
@@ -54,7 +60,9 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     W = 0x10000  # a fake, 16-byte aligned address: validation must fail before it is touched
     # bad descriptors
     assert E(None, W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(fmt=3)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=4)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=3, entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
+             None) == 1
     assert E(ctypes.byref(_desc(entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
     assert E(ctypes.byref(_desc(anchor=float("nan"))), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
     assert E(ctypes.byref(_desc(anchor=0.0)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
@@ -79,5 +87,9 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert lib.iq_decode(ctypes.byref(d), None, 4, 1, W, None) == 1
     assert lib.iq_choice_search(ctypes.byref(d), W, 0, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 2
     assert lib.iq_choice_search(ctypes.byref(d), W, 4, 2, 256, W, W, 2, 0, W, W, 2, None, None) == 1
+    # IQ1_M: any anchor (it is derived per block); no choice search
+    m = _desc(fmt=3, anchor=float("nan"))
+    assert E(ctypes.byref(m), W, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
+    assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 4
     assert lib.iq_sqrt_diag(None, 1, W, None) == 1
     assert lib.iq_sqrt_diag(W, 0, W, None) == 2
