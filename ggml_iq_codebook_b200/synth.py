@@ -27,6 +27,7 @@ BLOCK = 256
 
 IQ1S_GRID_ENTRIES = 2048
 IQ2XS_GRID_ENTRIES = 512
+IQ2S_GRID_ENTRIES = 1024
 
 
 def _distinct_rows(values: np.ndarray, n: int, seed: int) -> np.ndarray:
@@ -55,6 +56,11 @@ def iq1s_grid(seed: int = GRID_SEED) -> np.ndarray:
 def iq2xs_grid(seed: int = GRID_SEED + 1) -> np.ndarray:
     """[512, 8] int8, entries in {1, 3, 5, 7}, all rows distinct."""
     return _distinct_rows(np.array([1, 3, 5, 7], dtype=np.int8), IQ2XS_GRID_ENTRIES, seed)
+
+
+def iq2s_grid(seed: int = GRID_SEED + 2) -> np.ndarray:
+    """[1024, 8] int8, entries in {1, 3, 5, 7}, all rows distinct."""
+    return _distinct_rows(np.array([1, 3, 5, 7], dtype=np.int8), IQ2S_GRID_ENTRIES, seed)
 
 
 def normal_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:

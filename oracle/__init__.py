@@ -1,6 +1,6 @@
 """CPU oracle for the GGML IQ encoder path -- TEST INFRASTRUCTURE ONLY.
 
-A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS encoder and decoder,
+A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS / IQ2_S encoder and decoder,
 and the local-Hessian choice search (IQ1_S, IQ2_XS), with this thin ctypes wrapper. It is the yardstick the CUDA library is
 checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import it; the library never does, and the two share no code.
@@ -22,10 +22,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "iq_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-FMT = {"iq1_s": 1, "iq2_xs": 2, "iq1_m": 3}
-BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74, "iq1_m": 56}
-CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16, "iq1_m": 16}
-CHOICES = {"iq1_s": 16, "iq2_xs": 16, "iq1_m": 8}
+FMT = {"iq1_s": 1, "iq2_xs": 2, "iq1_m": 3, "iq2_s": 4}
+BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74, "iq1_m": 56, "iq2_s": 82}
+CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16, "iq1_m": 16, "iq2_s": 16}
+CHOICES = {"iq1_s": 16, "iq2_xs": 16, "iq1_m": 8, "iq2_s": 16}
 NUM_CHOICES = 16
 
 FLAG_NONFINITE = 1

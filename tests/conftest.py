@@ -21,9 +21,10 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def grids():
     from ggml_iq_codebook_b200 import synth
-    return {"iq1_s": synth.iq1s_grid(), "iq2_xs": synth.iq2xs_grid()}
+    return {"iq1_s": synth.iq1s_grid(), "iq2_xs": synth.iq2xs_grid(), "iq1_m": synth.iq1s_grid(),
+            "iq2_s": synth.iq2s_grid()}
 
 
 @pytest.fixture(scope="session")
 def anchors():
-    return {"iq1_s": IQ1S_ANCHOR, "iq2_xs": IQ2XS_ANCHOR}
+    return {"iq1_s": IQ1S_ANCHOR, "iq2_xs": IQ2XS_ANCHOR, "iq1_m": 1.0, "iq2_s": IQ2XS_ANCHOR}
