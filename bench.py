@@ -50,7 +50,8 @@ L2_FLUSH_BYTES = 256 << 20
 #     16 groups x 16 choices x (256 + 5 x 16 - 1) gains; gradient updates after a switch are
 #     data dependent and not counted: 310,528 ops.
 #   IQ1_M runs IQ1_S's search (same 2048 x 16 candidates per group): 2,949,120 ops per block.
-OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120}
+#   IQ2_S runs IQ2_XS's per-entry work over 1024 entries: 32 x 1024 x 48 = 1,572,864 per block.
+OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120, "iq2_s": 1_572_864}
 CHOICE_OPS_PER_ROW_BLOCK = 310_528
 SMS, FP32_LANES = 148, 128
 
@@ -164,8 +165,9 @@ class Workload:
         self.name, self.dev, self.peaks = name, dev, peaks
         g1 = torch.from_numpy(synth.iq1s_grid()).to(dev)
         g2 = torch.from_numpy(synth.iq2xs_grid()).to(dev)
+        g3 = torch.from_numpy(synth.iq2s_grid()).to(dev)
         self.desc = {"iq1_s": iq.make_desc("iq1_s", g1), "iq2_xs": iq.make_desc("iq2_xs", g2),
-                     "iq1_m": iq.make_desc("iq1_m", g1)}
+                     "iq1_m": iq.make_desc("iq1_m", g1), "iq2_s": iq.make_desc("iq2_s", g3)}
         self.launches_per_step = 2
         if name == "iq1s_4096x4096_weighted":
             wl = synth.workload_iq1s_4096x4096_weighted()
@@ -175,6 +177,10 @@ class Workload:
             wl = dict(synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m")
             self._encode_decode(wl, "IQ1_M importance-weighted encode + bf16 decode, 4096x4096 bf16 "
                                     "N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))")
+        elif name == "iq2s_8192x4096":
+            wl = dict(synth.workload_iq2xs_8192x4096(), fmt="iq2_s")
+            self._encode_decode(wl, "IQ2_S importance-weighted encode + bf16 decode, 8192x4096 bf16 "
+                                    "N(0,0.015^2), importance lognormal(0,1)")
         elif name == "iq2xs_8192x4096":
             wl = synth.workload_iq2xs_8192x4096()
             self._encode_decode(wl, "IQ2_XS importance-weighted encode + bf16 decode, 8192x4096 bf16 "
@@ -216,7 +222,7 @@ class Workload:
         self.units = self.w.numel()
         self.nblocks = self.units // 256
         self.text = text
-        self.dominant = "iq2xs_encode_kernel" if self.fmt == "iq2_xs" else "iq1_encode_kernel"
+        self.dominant = "iq2_encode_kernel" if self.fmt in ("iq2_xs", "iq2_s") else "iq1_encode_kernel"
         self.ops_per_launch = self.nblocks * OPS_PER_BLOCK[self.fmt]
         # validate once (findings word + raise) before anything is timed
         iq.iq_encode(self.desc[self.fmt], self.w, self.imp, out=self.payload)
@@ -367,9 +373,11 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
                   "iq1m_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
                   "iq1s_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
                   "iq2xs_8192x4096": synth.workload_iq2xs_8192x4096,
+                  "iq2s_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq1s_64x256": synth.workload_iq1s_64x256}[name]()
-            w, imp, fmt = wl["w"], wl["importance"], ("iq1_m" if name.startswith("iq1m") else wl["fmt"])
-        g = synth.iq2xs_grid() if fmt == "iq2_xs" else synth.iq1s_grid()
+            fmt = "iq1_m" if name.startswith("iq1m") else "iq2_s" if name.startswith("iq2s") else wl["fmt"]
+            w, imp = wl["w"], wl["importance"]
+        g = {"iq2_xs": synth.iq2xs_grid, "iq2_s": synth.iq2s_grid}.get(fmt, synth.iq1s_grid)()
 
         def run(r):
             p, _ = oracle.encode(fmt, g, iq.DEFAULT_ANCHOR[fmt], w[:r], importance=imp)

@@ -17,16 +17,16 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libiq_b200.so")
 
-IQ_FMT = {"iq1_s": 1, "iq2_xs": 2, "iq1_m": 3}
-BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74, "iq1_m": 56}
-CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16, "iq1_m": 16}
-GRID_ENTRIES = {"iq1_s": 2048, "iq2_xs": 512, "iq1_m": 2048}
-CHOICES = {"iq1_s": 16, "iq2_xs": 16, "iq1_m": 8}
+IQ_FMT = {"iq1_s": 1, "iq2_xs": 2, "iq1_m": 3, "iq2_s": 4}
+BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74, "iq1_m": 56, "iq2_s": 82}
+CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16, "iq1_m": 16, "iq2_s": 16}
+GRID_ENTRIES = {"iq1_s": 2048, "iq2_xs": 512, "iq1_m": 2048, "iq2_s": 1024}
+CHOICES = {"iq1_s": 16, "iq2_xs": 16, "iq1_m": 8, "iq2_s": 16}
 NUM_CHOICES = 16
 # d = fp16(fp32(amax / qmax) * anchor): IQ1_S's 0.61 is the pages' constant; IQ2_XS's was fixed
 # once by a seeded sweep on non-evaluation data (the pages name a clamp but give no numbers).
 # IQ1_M ignores the descriptor's anchor: it follows each block's peak-to-RMS.
-DEFAULT_ANCHOR = {"iq1_s": 0.61, "iq2_xs": 0.9, "iq1_m": 1.0}
+DEFAULT_ANCHOR = {"iq1_s": 0.61, "iq2_xs": 0.9, "iq1_m": 1.0, "iq2_s": 0.9}
 
 IQ_OUT_F32, IQ_OUT_BF16 = 0, 1
 FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
@@ -106,7 +106,7 @@ def make_desc(fmt: str, grid: torch.Tensor, anchor: float | None = None) -> IQDe
 
 
 def _fmt_of(desc: IQDesc) -> str:
-    return {1: "iq1_s", 2: "iq2_xs", 3: "iq1_m"}[desc.fmt]
+    return {1: "iq1_s", 2: "iq2_xs", 3: "iq1_m", 4: "iq2_s"}[desc.fmt]
 
 
 def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = None,
@@ -116,8 +116,8 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
     """Encode bf16 weights [rows, cols] or [batch, rows, cols] (last dim contiguous).
 
     importance: fp32 [cols] or [batch, cols]; choices: uint8 [..., rows, cols/256, G].
-    scales: static block scales, either fp16 [..., rows, cols/256] (contiguous) or, for IQ1_S and
-    IQ2_XS, an existing payload uint8 [..., rows, cols/256, B] whose d fields are read in place.
+    scales: static block scales, either fp16 [..., rows, cols/256] (contiguous) or, except for
+    IQ1_M, an existing payload uint8 [..., rows, cols/256, B] whose d fields are read in place.
     Returns the payload uint8 [(C,) (batch,) rows, cols/256, B], C = CHOICES[fmt]. With
     raise_on_flags (default) the call synchronises and raises on a device-side finding; pass a flags tensor and
     raise_on_flags=False to stay asynchronous, or flags=False to skip the findings word

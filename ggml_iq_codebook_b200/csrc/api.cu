@@ -41,6 +41,8 @@ iq_status check_desc(const iq_desc* d) {
         if (d->grid_entries != 2048) return IQ_EINVAL;
     } else if (d->fmt == IQ_FMT_IQ2_XS) {
         if (d->grid_entries != 512) return IQ_EINVAL;
+    } else if (d->fmt == IQ_FMT_IQ2_S) {
+        if (d->grid_entries != 1024) return IQ_EINVAL;
     } else {
         return IQ_EINVAL;
     }
@@ -57,15 +59,15 @@ iq_status launched(cudaError_t e) { return e == cudaSuccess ? IQ_OK : IQ_ECUDA; 
 extern "C" {
 
 size_t iq_block_bytes(int32_t fmt) {
-    return fmt == IQ_FMT_IQ1_S ? 50 : fmt == IQ_FMT_IQ2_XS ? 74 : fmt == IQ_FMT_IQ1_M ? 56 : 0;
+    return fmt == IQ_FMT_IQ1_S ? 50 : fmt == IQ_FMT_IQ2_XS ? 74 : fmt == IQ_FMT_IQ1_M ? 56 : fmt == IQ_FMT_IQ2_S ? 82 : 0;
 }
 
 int32_t iq_choice_groups(int32_t fmt) {
-    return fmt == IQ_FMT_IQ1_S ? 8 : (fmt == IQ_FMT_IQ2_XS || fmt == IQ_FMT_IQ1_M) ? 16 : 0;
+    return fmt == IQ_FMT_IQ1_S ? 8 : (fmt == IQ_FMT_IQ2_XS || fmt == IQ_FMT_IQ1_M || fmt == IQ_FMT_IQ2_S) ? 16 : 0;
 }
 
 int32_t iq_num_choices(int32_t fmt) {
-    return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS) ? 16 : fmt == IQ_FMT_IQ1_M ? 8 : 0;
+    return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS || fmt == IQ_FMT_IQ2_S) ? 16 : fmt == IQ_FMT_IQ1_M ? 8 : 0;
 }
 
 iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64_t rows, int64_t cols,
@@ -107,8 +109,9 @@ iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64
     p.anchor = desc->anchor;
     p.nb = batch * rows * (cols / 256);
     const int mode = every_choice ? iqk::kEvery : (choices != nullptr ? iqk::kFixed : iqk::kSearch);
-    return launched(desc->fmt == IQ_FMT_IQ2_XS ? iqk::launch_iq2xs_encode(p, mode, sms, stream)
-                                               : iqk::launch_iq1_encode(desc->fmt, p, mode, sms, stream));
+    const bool iq2 = desc->fmt == IQ_FMT_IQ2_XS || desc->fmt == IQ_FMT_IQ2_S;
+    return launched(iq2 ? iqk::launch_iq2_encode(desc->fmt, p, mode, sms, stream)
+                        : iqk::launch_iq1_encode(desc->fmt, p, mode, sms, stream));
 }
 
 iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks, int32_t out_dtype,
@@ -135,7 +138,7 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
                            int64_t payload_ld, uint32_t* flags, cudaStream_t stream) {
     iq_status st = check_desc(desc);
     if (st != IQ_OK) return st;
-    if (desc->fmt == IQ_FMT_IQ1_M) return IQ_EUNSUPPORTED;
+    if (desc->fmt != IQ_FMT_IQ1_S && desc->fmt != IQ_FMT_IQ2_XS) return IQ_EUNSUPPORTED;
     if (w == nullptr || hess == nullptr || cand == nullptr || picks == nullptr || payload == nullptr)
         return IQ_EINVAL;
     if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;

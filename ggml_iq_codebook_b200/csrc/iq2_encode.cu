@@ -1,4 +1,4 @@
-// iq2xs_encode.cu -- IQ2_XS encoder: sign parity + weighted exhaustive magnitude search + pack.
+// iq2_encode.cu -- IQ2_XS and IQ2_S encoders: weighted exhaustive magnitude search + pack.
 //
 // Method (PR #2450 review comments; IQ2_S codec commit text on the PR #2525 page): 32 groups of
 // 8 weights per 256-weight block, each coded as a 9-bit index into a 512 x 8 magnitude grid plus
@@ -13,6 +13,11 @@
 //           B = V_0 g_0,  then B = fma(V_j, g_j, B);   m = fma(s, A, B)
 //   argmin_g m (lowest entry on ties); e = s m_min; sub-block E = e_even + e_odd; argmin_ls E.
 //
+// IQ2_S (PR #2512 codec, PR #2565 CUDA encoder commit texts): a 1024-entry grid and a full 8-bit
+// sign mask per group, so the input's signs are kept (nothing is flipped) and a_j = |x_j|; the
+// 82-byte block holds d, the low index bytes, the sign bytes, the 2-bit high index fields (group
+// g at shift 2 (g % 4) of byte 66 + g/4) and the scale nibbles at bytes 74..81.
+//
 // Kernel design (B200): one warp per block, one lane per group; the 512-entry loop is warp-uniform
 // and reads each entry's 8 magnitudes and 8 squares (64 B) with broadcast 16-byte shared-memory
 // loads. Argmin bookkeeping as in the IQ1_S kernel: running minima, chunk of first appearance,
@@ -25,8 +30,15 @@ namespace iqk {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kFloatGridBytes = kIq2xsEntries * 16 * 4;  // per entry: g[8] then g^2[8] as fp32
-constexpr int kSmemBytes = kFloatGridBytes + kIq2xsEntries * 8;  // + the packed int8 grid
+
+template <int FMT>
+struct Iq2Cfg {
+    static constexpr bool S = FMT == IQ_FMT_IQ2_S;
+    static constexpr int E = S ? kIq2sEntries : kIq2xsEntries;
+    static constexpr int BYTES = S ? kIq2sBytes : kIq2xsBytes;
+    static constexpr int FLOAT_GRID_BYTES = E * 16 * 4;           // per entry: g[8] then g^2[8] as fp32
+    static constexpr int SMEM = FLOAT_GRID_BYTES + E * 8;         // + the packed int8 grid
+};
 
 struct Entry {
     float g[8], gg[8];
@@ -62,8 +74,9 @@ __device__ __forceinline__ void entry_AB(const Entry& en, const float w[8], cons
     }
 }
 
+template <int BYTES>
 __device__ __forceinline__ void write_zero_block(uint8_t* out, int lane) {
-    for (int i = lane; i < kIq2xsBytes / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
+    for (int i = lane; i < BYTES / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
 }
 
 // lane = group: code = idx | sign7 << 9; ls = its sub-block's local scale.
@@ -76,15 +89,39 @@ __device__ __forceinline__ void pack_block(uint8_t* out, int lane, int idx, uint
     if (lane == 0) *reinterpret_cast<uint16_t*>(out) = d_half;
 }
 
-template <int MODE, int K>
-__global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const EncodeParams p) {
+// IQ2_S: lane = group: low index byte, sign byte, 2 high index bits (4 groups per byte), and the
+// sub-block's scale nibble.
+__device__ __forceinline__ void pack_block_s(uint8_t* out, int lane, int idx, uint32_t neg, int ls,
+                                             uint16_t d_half) {
+    out[2 + lane] = static_cast<uint8_t>(idx & 0xFF);
+    out[34 + lane] = static_cast<uint8_t>(neg);
+    uint32_t v = static_cast<uint32_t>((idx >> 8) & 3) << (2 * (lane & 3));
+    v |= __shfl_xor_sync(0xffffffffu, v, 1);
+    v |= __shfl_xor_sync(0xffffffffu, v, 2);
+    const int hi = __shfl_down_sync(0xffffffffu, ls, 2);  // sub-block 2i+1 sits 2 lanes up
+    if ((lane & 3) == 0) {
+        out[66 + (lane >> 2)] = static_cast<uint8_t>(v);
+        out[74 + (lane >> 2)] = static_cast<uint8_t>(ls | (hi << 4));
+    }
+    if (lane == 0) *reinterpret_cast<uint16_t*>(out) = d_half;
+}
+
+template <int FMT>
+__device__ __forceinline__ void pack(uint8_t* out, int lane, int idx, uint32_t neg, int ls, uint16_t d_half) {
+    if (Iq2Cfg<FMT>::S) pack_block_s(out, lane, idx, neg, ls, d_half);
+    else pack_block(out, lane, idx, neg, ls, d_half);
+}
+
+template <int FMT, int MODE, int K>
+__global__ void __launch_bounds__(kWarps * 32, 2) iq2_encode_kernel(const EncodeParams p) {
+    using Cfg = Iq2Cfg<FMT>;
     extern __shared__ __align__(16) char smem[];
     float* sgf = reinterpret_cast<float*>(smem);
     const float4* sg = reinterpret_cast<const float4*>(smem);
-    int2* sgp = reinterpret_cast<int2*>(smem + kFloatGridBytes);
+    int2* sgp = reinterpret_cast<int2*>(smem + Cfg::FLOAT_GRID_BYTES);
 
     bool bad = false;
-    for (int q = threadIdx.x; q < kIq2xsEntries; q += blockDim.x) {
+    for (int q = threadIdx.x; q < Cfg::E; q += blockDim.x) {
         const int2 raw = __ldg(reinterpret_cast<const int2*>(p.grid) + q);
         sgp[q] = raw;
 #pragma unroll
@@ -105,8 +142,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
     for (int64_t b = static_cast<int64_t>(blockIdx.x) * kWarps + warp; b < p.nb; b += stride) {
         const int64_t e = b / per_batch, rem = b - e * per_batch;
         const int64_t r = rem / p.nblk, blk = rem - r * p.nblk;
-        uint8_t* out = p.payload + b * kIq2xsBytes;
-        const int64_t every_stride = p.nb * kIq2xsBytes;
+        uint8_t* out = p.payload + b * Cfg::BYTES;
+        const int64_t every_stride = p.nb * Cfg::BYTES;
 
         float x[8], w[8];
         unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(p.w + e * p.w_bstride + r * p.ldw + blk * kBlock) + lane), x);
@@ -143,9 +180,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
         }
         if (f != 0 || bad || (d_half & 0x7FFFu) == 0) {
             if (MODE == kEvery) {
-                for (int c = 0; c < kChoices; ++c) write_zero_block(out + c * every_stride, lane);
+                for (int c = 0; c < kChoices; ++c) write_zero_block<Cfg::BYTES>(out + c * every_stride, lane);
             } else {
-                write_zero_block(out, lane);
+                write_zero_block<Cfg::BYTES>(out, lane);
             }
             if (lane == 0) raise_flags(p.flags, f);
             continue;
@@ -157,7 +194,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
 #pragma unroll
         for (int j = 0; j < 8; ++j) neg |= static_cast<uint32_t>(x[j] < 0.0f) << j;
         int flipped = -1;
-        if (__popc(neg) & 1) {
+        if (!Cfg::S && (__popc(neg) & 1)) {
             int k = 0;
             float tk = __fmul_rn(__fmul_rn(x[0], x[0]), w[0]);
 #pragma unroll
@@ -185,7 +222,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
             float best = INFINITY;
             int bi = 0;
 #pragma unroll 2
-            for (int q = 0; q < kIq2xsEntries; ++q) {
+            for (int q = 0; q < Cfg::E; ++q) {
                 Entry en;
                 load_entry(sg, q, en);
                 float A, B;
@@ -193,7 +230,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
                 const float m = __fmaf_rn(sv, A, B);
                 if (m < best) { best = m; bi = q; }
             }
-            pack_block(out, lane, bi, neg, fixed_c, d_half);
+            pack<FMT>(out, lane, bi, neg, fixed_c, d_half);
             continue;
         }
 
@@ -201,7 +238,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
         int bch[kChoices];
 #pragma unroll
         for (int c = 0; c < kChoices; ++c) { best[c] = INFINITY; bch[c] = 0; }
-        for (int ch = 0; ch < kIq2xsEntries / K; ++ch) {
+        for (int ch = 0; ch < Cfg::E / K; ++ch) {
             float cm[kChoices];
             {
                 Entry ea, eb;
@@ -248,7 +285,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
         };
 
         if (MODE == kEvery) {
-            for (int c = 0; c < kChoices; ++c) pack_block(out + c * every_stride, lane, entry_of(c), neg, c, d_half);
+            for (int c = 0; c < kChoices; ++c) pack<FMT>(out + c * every_stride, lane, entry_of(c), neg, c, d_half);
             continue;
         }
 
@@ -260,30 +297,37 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2xs_encode_kernel(const Enco
             const float E = __fadd_rn(e0, __shfl_xor_sync(0xffffffffu, e0, 1));
             if (E < bestE) { bestE = E; cstar = c; }
         }
-        pack_block(out, lane, entry_of(cstar), neg, cstar, d_half);
+        pack<FMT>(out, lane, entry_of(cstar), neg, cstar, d_half);
     }
 }
 
-template <int MODE, int K>
+template <int FMT, int MODE, int K>
 cudaError_t launch_mode(const EncodeParams& p, int num_sms, cudaStream_t s) {
-    auto kern = iq2xs_encode_kernel<MODE, K>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    constexpr int smem = Iq2Cfg<FMT>::SMEM;
+    auto kern = iq2_encode_kernel<FMT, MODE, K>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     const int64_t ctas_needed = (p.nb + kWarps - 1) / kWarps;
     const int64_t ctas = ctas_needed < 2LL * num_sms ? ctas_needed : 2LL * num_sms;
-    kern<<<static_cast<unsigned>(ctas), kWarps * 32, kSmemBytes, s>>>(p);
+    kern<<<static_cast<unsigned>(ctas), kWarps * 32, smem, s>>>(p);
     return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const EncodeParams& p, int mode, int num_sms, cudaStream_t s) {
+    switch (mode) {
+        case kSearch: return launch_mode<FMT, kSearch, 32>(p, num_sms, s);
+        case kFixed: return launch_mode<FMT, kFixed, 32>(p, num_sms, s);
+        default: return launch_mode<FMT, kEvery, 8>(p, num_sms, s);
+    }
 }
 
 }  // namespace
 
-cudaError_t launch_iq2xs_encode(const EncodeParams& p, int mode, int num_sms, cudaStream_t s) {
+cudaError_t launch_iq2_encode(int fmt, const EncodeParams& p, int mode, int num_sms, cudaStream_t s) {
     if (p.nb == 0) return cudaSuccess;
-    switch (mode) {
-        case kSearch: return launch_mode<kSearch, 32>(p, num_sms, s);
-        case kFixed: return launch_mode<kFixed, 32>(p, num_sms, s);
-        default: return launch_mode<kEvery, 8>(p, num_sms, s);
-    }
+    return fmt == IQ_FMT_IQ2_S ? launch_fmt<IQ_FMT_IQ2_S>(p, mode, num_sms, s)
+                               : launch_fmt<IQ_FMT_IQ2_XS>(p, mode, num_sms, s);
 }
 
 }  // namespace iqk

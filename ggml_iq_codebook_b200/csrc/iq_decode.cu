@@ -1,4 +1,4 @@
-// iq_decode.cu -- IQ1_S / IQ2_XS / IQ1_M decoders (sm_100a), HBM-bound.
+// iq_decode.cu -- IQ1_S / IQ2_XS / IQ1_M / IQ2_S decoders (sm_100a), HBM-bound.
 //
 // Values (PR #2450 review comments):
 //   IQ1_S  x = d (2 ls + 1) (q_j + delta), index = low | ((qh >> 3i) & 7) << 8, ls = qh bits
@@ -8,6 +8,8 @@
 //   IQ1_M  (PR #2513) x = d (2 ls + 1) (q_j + delta), d = the top nibbles of the four scale words
 //          at bytes 48..55, ls of choice group k = bits 3(k%4).. of word k/4, group g's index
 //          = byte g | (nibble g of bytes 32.. & 7) << 8, delta = -1/8 if that nibble's bit 3.
+//   IQ2_S  (PR #2512) x = d (2 ls + 1) g_j (-1)^sign_j, index = byte 2 + g | 2 bits at shift
+//          2 (g % 4) of byte 66 + g/4 << 8, sign mask = byte 34 + g, ls as IQ2_XS at bytes 74...
 // Every value is a product of at most 20 significant bits, so the fp32 result is exact; the bf16
 // output is its round-to-nearest-even. Each block decodes independently, so the output does not
 // depend on how a caller chunks the blocks.
@@ -112,6 +114,29 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
         return;
     }
     const float d = half_bits_to_f32(pw[0]);
+    if (FMT == IQ_FMT_IQ2_S) {
+        const uint32_t sc = pb[74 + (h >> 1)];
+        const int ls = static_cast<int>((h & 1) ? (sc >> 4) : (sc & 15u));
+        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
+        const uint32_t lw = pw[1 + h];                  // low index bytes of groups 2h, 2h + 1
+        const uint32_t sg = pw[17 + h];                 // their sign bytes
+        const uint32_t hb = pb[66 + (h >> 1)] >> (4 * (h & 1));
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t idx = ((lw >> (8 * t)) & 0xFFu) | (((hb >> (2 * t)) & 3u) << 8);
+            const uint32_t neg = (sg >> (8 * t)) & 0xFFu;
+            const uint32_t e = sgrid[idx];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t cj = (e >> (2 * j)) & 3u;
+                const float a = (cj & 2u) ? ((cj & 1u) ? m7 : m5) : ((cj & 1u) ? m3 : m1);
+                v[8 * t + j] = ((neg >> j) & 1u) ? -a : a;
+            }
+        }
+        store16<BF16>(out, b * 32 + 2 * h, v);
+        return;
+    }
     if (FMT == IQ_FMT_IQ1_S) {
         const uint32_t lw = pw[1 + h];          // low index bytes of groups 2h, 2h + 1
         const uint32_t qh = pw[17 + (h >> 1)];  // the sub-block's qh
@@ -153,8 +178,12 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
 
 template <int FMT>
 struct DecodeCfg {
-    static constexpr int BYTES = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : FMT == IQ_FMT_IQ1_M ? kIq1mBytes : kIq2xsBytes;
-    static constexpr int E = FMT == IQ_FMT_IQ2_XS ? kIq2xsEntries : kIq1sEntries;
+    static constexpr int BYTES = FMT == IQ_FMT_IQ1_S   ? kIq1sBytes
+                                 : FMT == IQ_FMT_IQ1_M ? kIq1mBytes
+                                 : FMT == IQ_FMT_IQ2_S ? kIq2sBytes
+                                                       : kIq2xsBytes;
+    static constexpr bool IQ2 = FMT == IQ_FMT_IQ2_XS || FMT == IQ_FMT_IQ2_S;
+    static constexpr int E = FMT == IQ_FMT_IQ2_XS ? kIq2xsEntries : FMT == IQ_FMT_IQ2_S ? kIq2sEntries : kIq1sEntries;
     static constexpr int TILE_BYTES = kTileBlocks * BYTES;  // a multiple of 16
     static constexpr int GRID_BYTES = (E * 2 + 15) / 16 * 16;
     static constexpr int smem = GRID_BYTES + 2 * TILE_BYTES;
@@ -168,7 +197,7 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
-        if (FMT != IQ_FMT_IQ2_XS) c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
+        if (!DecodeCfg<FMT>::IQ2) c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
         else c |= (static_cast<uint32_t>((v - 1) >> 1) & 3u) << (2 * j);
     }
     return static_cast<uint16_t>(c);
@@ -237,6 +266,7 @@ cudaError_t launch_decode(int fmt, bool bf16, const DecodeParams& p, int num_sms
     if (p.nblocks == 0) return cudaSuccess;
     if (fmt == IQ_FMT_IQ1_S) return bf16 ? launch<IQ_FMT_IQ1_S, true>(p, num_sms, s) : launch<IQ_FMT_IQ1_S, false>(p, num_sms, s);
     if (fmt == IQ_FMT_IQ1_M) return bf16 ? launch<IQ_FMT_IQ1_M, true>(p, num_sms, s) : launch<IQ_FMT_IQ1_M, false>(p, num_sms, s);
+    if (fmt == IQ_FMT_IQ2_S) return bf16 ? launch<IQ_FMT_IQ2_S, true>(p, num_sms, s) : launch<IQ_FMT_IQ2_S, false>(p, num_sms, s);
     return bf16 ? launch<IQ_FMT_IQ2_XS, true>(p, num_sms, s) : launch<IQ_FMT_IQ2_XS, false>(p, num_sms, s);
 }
 

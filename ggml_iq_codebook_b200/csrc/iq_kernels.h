@@ -45,7 +45,7 @@ struct ChoiceParams {
 
 // Each returns the cudaError_t of its launch (cudaSuccess when nothing had to run).
 cudaError_t launch_iq1_encode(int fmt, const EncodeParams& p, int mode, int num_sms, cudaStream_t s);
-cudaError_t launch_iq2xs_encode(const EncodeParams& p, int mode, int num_sms, cudaStream_t s);
+cudaError_t launch_iq2_encode(int fmt, const EncodeParams& p, int mode, int num_sms, cudaStream_t s);
 cudaError_t launch_decode(int fmt, bool bf16, const DecodeParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_choice_search(int fmt, const ChoiceParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t s);

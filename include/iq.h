@@ -14,7 +14,9 @@
  *   - fixed per-group choices (PR #3157) and the one-pass every-choice encode (PR #3159);
  *   - IQ1_M (PR #2513 codec and PR #2595 encoder commit texts): the IQ1_S search with a local
  *     scale per 16 weights, a delta per 8-weight group and d kept in four scale words;
- *   - decoding of the three layouts;
+ *   - IQ2_S (PR #2512 codec and PR #2565 encoder commit texts): the IQ2_XS search over a
+ *     1024-entry grid with a full 8-bit sign mask per group (the input's signs, no parity flip);
+ *   - decoding of the four layouts;
  *   - the local-Hessian choice search (PR #3158, fused in PR #3218 "[4/4] Run the local-Hessian
  *     choice search as one CUDA kernel").
  *
@@ -54,7 +56,7 @@ typedef enum {
     IQ_EUNSUPPORTED = 4   /* the current device is not sm_100, or the call does not take the format */
 } iq_status;
 
-typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3 } iq_format;
+typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3, IQ_FMT_IQ2_S = 4 } iq_format;
 
 typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 
@@ -67,15 +69,15 @@ typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 
 /*
  * Codebook/convention descriptor (host struct; the grid it points to lives on the device).
- *   fmt           IQ_FMT_IQ1_S, IQ_FMT_IQ2_XS or IQ_FMT_IQ1_M
- *   grid_entries  2048 (IQ1_S, IQ1_M) or 512 (IQ2_XS)
+ *   fmt           IQ_FMT_IQ1_S, IQ_FMT_IQ2_XS, IQ_FMT_IQ1_M or IQ_FMT_IQ2_S
+ *   grid_entries  2048 (IQ1_S, IQ1_M), 512 (IQ2_XS) or 1024 (IQ2_S)
  *   grid          device int8 [grid_entries][8]; IQ1_S and IQ1_M values in {-1,0,1} (a ternary
- *                 grid, PR #2723; IQ1_M shares IQ1_S's, PR #2513), IQ2_XS magnitudes in {1,3,5,7}.
+ *                 grid, PR #2723; IQ1_M shares IQ1_S's, PR #2513), IQ2_XS and IQ2_S magnitudes in {1,3,5,7}.
  *                 Row q, column j multiplies weight j of a group.
  *   anchor        the scale predictor's anchor: d = fp16(fp32(amax / qmax) * anchor), with
  *                 qmax = 16.875 (IQ1_S, = 15 * 1.125, the largest |s (q + delta)| in units of d)
- *                 and 217 (IQ2_XS, = 31 * 7). IQ1_S uses 0.61 (PR #2450 review). The pages give
- *                 no IQ2_XS constant; this library's default is 0.9. IQ1_M ignores it: its anchor
+ *                 and 217 (IQ2_XS and IQ2_S, = 31 * 7). IQ1_S uses 0.61 (PR #2450 review). The
+ *                 pages give no IQ2_XS or IQ2_S constant; this library's default is 0.9. IQ1_M ignores it: its anchor
  *                 is clamp(0.58 + 0.035 * amax / rms, 0.65, 0.95) per block (PR #2513), rms over
  *                 the block's 256 weights (squares summed per 8-weight group in order, the 32
  *                 group sums by a pairwise tree), with qmax = 16.875.
@@ -87,16 +89,17 @@ typedef struct {
     float anchor;
 } iq_desc;
 
-/* Bytes per 256-weight block: 50 (IQ1_S), 74 (IQ2_XS), 56 (IQ1_M); 0 for an unknown format. */
+/* Bytes per 256-weight block: 50 (IQ1_S), 74 (IQ2_XS), 56 (IQ1_M), 82 (IQ2_S); 0 for an unknown
+ * format. */
 size_t iq_block_bytes(int32_t fmt);
 
 /* Choice groups per block: 8 (IQ1_S, one per 32 weights: local scale + delta sign),
- * 16 (IQ2_XS, one 4-bit local scale per 16 weights; IQ1_M, one 3-bit local scale per 16 weights,
- * each 8-weight group taking its own delta); 0 for an unknown format. */
+ * 16 (IQ2_XS and IQ2_S, one 4-bit local scale per 16 weights; IQ1_M, one 3-bit local scale per
+ * 16 weights, each 8-weight group taking its own delta); 0 for an unknown format. */
 int32_t iq_choice_groups(int32_t fmt);
 
-/* Choices per group: 16 for IQ1_S (c = ls + 8 * [delta < 0]) and IQ2_XS (c = ls); 8 for IQ1_M
- * (c = ls); 0 for an unknown format. */
+/* Choices per group: 16 for IQ1_S (c = ls + 8 * [delta < 0]), IQ2_XS and IQ2_S (c = ls); 8 for
+ * IQ1_M (c = ls); 0 for an unknown format. */
 int32_t iq_num_choices(int32_t fmt);
 
 /*
@@ -111,7 +114,8 @@ int32_t iq_num_choices(int32_t fmt);
  *     block's d (static scales, PR #3197, its "Static scales" item): block n of the flattened
  *     [batch][rows][cols/256] order takes d = scales[n * scales_stride] and is searched and packed
  *     under it whatever its amax. scales_stride >= 1 (uint16 elements): 1 for a dense array, or
- *     B/2 to read the d of an existing IQ1_S or IQ2_XS payload in place (its first two bytes).
+ *     B/2 to read the d of an existing IQ1_S, IQ2_XS or IQ2_S payload in place (its first two
+ *     bytes).
  *     A negative, infinite or NaN d gives the all-zero payload and IQ_FLAG_RANGE; d = +-0 gives
  *     the all-zero payload. Works with every mode.
  *   every_choice: 0, or 1 to write all C choices' payloads in one sweep (PR #3159):
@@ -129,7 +133,10 @@ int32_t iq_num_choices(int32_t fmt);
  *          the low nibble of byte 32+i): 3 high index bits, bit 3 set for delta = -1/8; 48..55
  *          four LE uint16 scale words: word i holds the 3-bit ls of choice groups 4i..4i+3 at
  *          shifts 0,3,6,9 and bits 12..15 of word i are bits 4i..4i+3 of fp16 d (PR #2513).
- * Value of a weight: IQ1_S, IQ1_M d (2 ls + 1)(q + delta); IQ2_XS d (2 ls + 1) g sign.
+ *   IQ2_S  bytes 0-1 fp16 d; 2..33 low 8 bits of the 32 group indices; 34..65 the groups' 8-bit
+ *          sign masks (bit j set: element j negative); 66..73 the 2 high index bits, group g at
+ *          shift 2 (g % 4) of byte 66 + g/4; 74..81 sixteen 4-bit local scales as IQ2_XS's.
+ * Value of a weight: IQ1_S, IQ1_M d (2 ls + 1)(q + delta); IQ2_XS, IQ2_S d (2 ls + 1) g sign.
  * IQ1_M picks, per group and ls, the (delta, entry) of least error, the lower shift (+1/8) and
  * then the lower entry on equal error (PR #2595); a choice group's error is the sum of its two
  * groups'.
@@ -154,7 +161,8 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
 
 /*
  * Local-Hessian choice search (PR #3158 steps; one fused launch as in PR #3218) for the first
- * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S and IQ2_XS (IQ1_M: IQ_EUNSUPPORTED).
+ * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S and IQ2_XS (other formats:
+ * IQ_EUNSUPPORTED).
  *   hess: fp32 [nblk][256][256], the symmetric diagonal block of the input Hessian per block,
  *     read as H[k][i] (row k, column i) for (H v)_i.
  *   cand: the every-choice payloads of those blocks; candidate c of (row r, block b) starts at

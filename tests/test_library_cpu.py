@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_format_tables(lib):
     assert lib.iq_block_bytes(1) == 50 and lib.iq_block_bytes(2) == 74 and lib.iq_block_bytes(3) == 56
-    assert lib.iq_block_bytes(4) == 0
+    assert lib.iq_block_bytes(4) == 82 and lib.iq_block_bytes(5) == 0
     assert lib.iq_choice_groups(1) == 8 and lib.iq_choice_groups(2) == 16 and lib.iq_choice_groups(3) == 16
     assert lib.iq_num_choices(1) == 16 and lib.iq_num_choices(2) == 16 and lib.iq_num_choices(3) == 8
     assert lib.iq_num_choices(0) == 0
@@ -60,7 +60,9 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     W = 0x10000  # a fake, 16-byte aligned address: validation must fail before it is touched
     # bad descriptors
     assert E(None, W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(fmt=4)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=5)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=4, entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
+             None) == 1
     assert E(ctypes.byref(_desc(fmt=3, entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
              None) == 1
     assert E(ctypes.byref(_desc(entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
@@ -91,5 +93,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     m = _desc(fmt=3, anchor=float("nan"))
     assert E(ctypes.byref(m), W, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
     assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 4
+    s2 = _desc(fmt=4, entries=1024, anchor=0.9)
+    assert lib.iq_choice_search(ctypes.byref(s2), W, 4, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 4
     assert lib.iq_sqrt_diag(None, 1, W, None) == 1
     assert lib.iq_sqrt_diag(W, 0, W, None) == 2
