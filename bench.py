@@ -45,14 +45,16 @@ L2_FLUSH_BYTES = 256 << 20
 #     per 256-weight block: 32 groups x 2048 entries x 45 = 2,949,120 ops.
 #   IQ2_XS, per (group, entry): A and B chains (16) + 16 x (fma + min) = 48 ops;
 #     per block: 32 x 512 x 48 = 786,432 ops.
-#   Choice search (IQ2_XS, 16 groups of 16 columns, 16 choices), per row and block:
-#     own-block scores 16 x 16 x (256 + 16 + 15), gradient 256 x 256, two sweeps of
-#     16 groups x 16 choices x (256 + 5 x 16 - 1) gains; gradient updates after a switch are
-#     data dependent and not counted: 310,528 ops.
+#   Choice search (G choice groups of W = 256 / G columns, 16 choices), per row and block:
+#     own-block scores G x 16 x (W^2 + 2W - 1), gradient 256 x 256, two sweeps of
+#     G x 16 x (W^2 + 5W - 1) gains; gradient updates after a switch are data dependent and not
+#     counted. IQ2_XS and IQ2_S (G = 16): 310,528 ops; IQ1_S (G = 8): 507,520 ops.
 #   IQ1_M runs IQ1_S's search (same 2048 x 16 candidates per group): 2,949,120 ops per block.
 #   IQ2_S runs IQ2_XS's per-entry work over 1024 entries: 32 x 1024 x 48 = 1,572,864 per block.
 OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120, "iq2_s": 1_572_864}
-CHOICE_OPS_PER_ROW_BLOCK = 310_528
+def choice_ops_per_row_block(G: int) -> int:
+    W = 256 // G
+    return G * 16 * (W * W + 2 * W - 1) + 256 * 256 + 2 * G * 16 * (W * W + 5 * W - 1)
 SMS, FP32_LANES = 148, 128
 
 
@@ -193,7 +195,11 @@ class Workload:
             wl = synth.workload_iq1s_64x256()
             self._encode_decode(wl, "IQ1_S encode + bf16 decode, one 64x256 bf16 weight, uniform importance")
         elif name == "choice_iq2xs_4096x4096":
-            self._choice(synth.workload_choice_iq2xs())
+            self._choice(synth.workload_choice_iq2xs(), "iq2_xs")
+        elif name == "choice_iq2s_4096x4096":
+            self._choice(synth.workload_choice_iq2xs(), "iq2_s")
+        elif name == "choice_iq1s_4096x4096":
+            self._choice(synth.workload_choice_iq2xs(), "iq1_s")
         elif name == "iq1s_decode_1m_blocks":
             wl = synth.workload_iq1s_4096x4096_weighted()
             self._encode_decode(wl, "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 weighted payload x16)")
@@ -227,25 +233,26 @@ class Workload:
         # validate once (findings word + raise) before anything is timed
         iq.iq_encode(self.desc[self.fmt], self.w, self.imp, out=self.payload)
 
-    def _choice(self, wl):
-        self.fmt, self.kind = "iq2_xs", "choice"
+    def _choice(self, wl, fmt):
+        self.fmt, self.kind = fmt, "choice"
         self.w_host, self.hess_host = wl["w"], wl["hess"]
         self.w, self.hess = wl["w"].to(self.dev), wl["hess"].to(self.dev)
         rows, cols = self.w.shape
         nblk = cols // 256
         self.imp = torch.empty(cols, dtype=torch.float32, device=self.dev)
-        self.cand = torch.empty((16, rows, nblk, 74), dtype=torch.uint8, device=self.dev)
-        self.picks = torch.empty((rows, nblk, 16), dtype=torch.uint8, device=self.dev)
-        self.payload = torch.empty((rows, nblk, 74), dtype=torch.uint8, device=self.dev)
+        B, G = iq.BLOCK_BYTES[fmt], iq.CHOICE_GROUPS[fmt]
+        self.cand = torch.empty((16, rows, nblk, B), dtype=torch.uint8, device=self.dev)
+        self.picks = torch.empty((rows, nblk, G), dtype=torch.uint8, device=self.dev)
+        self.payload = torch.empty((rows, nblk, B), dtype=torch.uint8, device=self.dev)
         self.units = self.w.numel()
         self.nblocks = rows * nblk
         self.launches_per_step = 3
-        self.text = ("local-Hessian choice search, IQ2_XS: sqrt(diag H) + one-pass every-choice encode + "
+        self.text = (f"local-Hessian choice search, {fmt.upper()}: sqrt(diag H) + one-pass every-choice encode + "
                      "two-sweep search, 4096x4096 bf16 N(0,0.02^2), 16 blocks of H = U^-1 U^-T")
         self.dominant = "choice_search_kernel"
-        self.ops_per_launch = rows * nblk * CHOICE_OPS_PER_ROW_BLOCK
+        self.ops_per_launch = rows * nblk * choice_ops_per_row_block(G)
         iq.iq_sqrt_diag(self.hess, out=self.imp)
-        iq.iq_encode(self.desc["iq2_xs"], self.w, self.imp, every_choice=True, out=self.cand)
+        iq.iq_encode(self.desc[fmt], self.w, self.imp, every_choice=True, out=self.cand)
 
     # one step; `ev` is a list of (start, end) event pairs to fill around the dominant kernel
     def step(self, ev=None):
@@ -354,15 +361,17 @@ def decode_roofline(wl: Workload, dev, peaks):
 def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None):
     """Oracle encode + decode on the first rows of the workload, sized to ~budget_s of wall time."""
     import oracle
-    if name == "choice_iq2xs_4096x4096":
+    if name.startswith("choice_"):
+        cfmt = {"choice_iq2xs_4096x4096": "iq2_xs", "choice_iq2s_4096x4096": "iq2_s",
+                "choice_iq1s_4096x4096": "iq1_s"}[name]
         wl = synth.workload_choice_iq2xs()
         w, hess = wl["w"], wl["hess"].numpy()
-        g = synth.iq2xs_grid()
+        g = {"iq2_xs": synth.iq2xs_grid, "iq2_s": synth.iq2s_grid, "iq1_s": synth.iq1s_grid}[cfmt]()
         imp = oracle.sqrt_diag(hess)
 
         def run(r):
-            cand, _ = oracle.encode("iq2_xs", g, iq.DEFAULT_ANCHOR["iq2_xs"], w[:r], importance=imp, every_choice=True)
-            oracle.choice_search("iq2_xs", g, w[:r], hess, cand)
+            cand, _ = oracle.encode(cfmt, g, iq.DEFAULT_ANCHOR[cfmt], w[:r], importance=imp, every_choice=True)
+            oracle.choice_search(cfmt, g, w[:r], hess, cand)
         cols = w.shape[1]
     else:
         if name == "iq1s_moe_256x1536x4096":

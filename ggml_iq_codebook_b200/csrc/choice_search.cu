@@ -13,7 +13,9 @@
 // all 256 k; sums over i inside a group are a pairwise tree; gain = fma(2, t1, t2); switching
 // updates grad_i by an fma chain over the group's k. NaN and +inf scores never win.
 //
-// Design (B200): one CTA = 16 (IQ2_XS) or 8 (IQ1_S) rows of one block, a half-warp per row and
+// Formats: IQ1_S (8 groups of 32 columns), IQ2_XS and IQ2_S (16 groups of 16 columns); 16 choices.
+//
+// Design (B200): one CTA = 16 (IQ2_XS, IQ2_S) or 8 (IQ1_S) rows of one block, a half-warp per row and
 // one lane per choice. The
 // rows run the group steps in lockstep, so each step stages one panel of H (the group's W rows,
 // W x 256 fp32) in shared memory once for all rows, double-buffered with cp.async so the next
@@ -41,8 +43,8 @@ __device__ __forceinline__ void load_vec(const float* src, float v[N]) {
     }
 }
 
-// The grid staged as 16-bit element codes: IQ1_S (+1 mask) | (-1 mask) << 8; IQ2_XS two bits
-// (g - 1) / 2 per element.
+// The grid staged as 16-bit element codes: IQ1_S (+1 mask) | (-1 mask) << 8; IQ2_XS and IQ2_S
+// two bits (g - 1) / 2 per element.
 template <int FMT>
 __device__ __forceinline__ uint16_t grid_code(int2 raw) {
     uint32_t c = 0;
@@ -62,7 +64,23 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
 template <int FMT>
 __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid, int g, int grp8, float xh[8]) {
     const float d = half_bits_to_f32(*reinterpret_cast<const uint16_t*>(pc));
-    if (FMT == IQ_FMT_IQ2_XS) {
+    if (FMT == IQ_FMT_IQ2_S) {
+        // 82-byte layout: low index byte 2 + grp8, sign byte 34 + grp8, 2 high index bits at
+        // shift 2 (grp8 % 4) of byte 66 + grp8 / 4, choice group g's scale nibble at 74 + g / 2
+        const uint32_t sc = pc[74 + (g >> 1)];
+        const int ls = static_cast<int>((g & 1) ? (sc >> 4) : (sc & 15u));
+        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
+        const uint32_t idx = static_cast<uint32_t>(pc[2 + grp8]) | (((static_cast<uint32_t>(pc[66 + (grp8 >> 2)]) >> (2 * (grp8 & 3))) & 3u) << 8);
+        const uint32_t neg = pc[34 + grp8];
+        const uint32_t e = sgrid[idx];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t cj = (e >> (2 * j)) & 3u;
+            const float a = (cj & 2u) ? ((cj & 1u) ? m7 : m5) : ((cj & 1u) ? m3 : m1);
+            xh[j] = ((neg >> j) & 1u) ? -a : a;
+        }
+    } else if (FMT == IQ_FMT_IQ2_XS) {
         const uint32_t code = *reinterpret_cast<const uint16_t*>(pc + 2 + 2 * grp8);
         const uint32_t sc = pc[66 + (g >> 1)];
         const int ls = static_cast<int>((g & 1) ? (sc >> 4) : (sc & 15u));
@@ -107,8 +125,8 @@ struct Cfg {
     static constexpr int RG = R / 4;                            // 4-row groups of the gradient tiles
     static constexpr int G = FMT == IQ_FMT_IQ1_S ? 8 : 16;     // choice groups per block
     static constexpr int W = kBlock / G;                        // columns per choice group
-    static constexpr int B = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : kIq2xsBytes;
-    static constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : kIq2xsEntries;
+    static constexpr int B = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : FMT == IQ_FMT_IQ2_S ? kIq2sBytes : kIq2xsBytes;
+    static constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : FMT == IQ_FMT_IQ2_S ? kIq2sEntries : kIq2xsEntries;
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
     // shared memory layout (bytes)
     static constexpr int oHp = 0;                                 // float [2][W][256], double buffer
@@ -383,6 +401,16 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
             uint8_t v;
             if (i < 2) {
                 v = cand[i];
+            } else if (FMT == IQ_FMT_IQ2_S) {
+                if (i < 66) {  // low index and sign bytes of 8-weight group q8: choice group q8 / 2
+                    v = cand[pick[((i - 2) & 31) >> 1] * C::B + i];
+                } else if (i < 74) {  // 2-bit high index fields: groups 4q, 4q+1 | 4q+2, 4q+3
+                    const int k = 2 * (i - 66);
+                    v = static_cast<uint8_t>((cand[pick[k] * C::B + i] & 0x0Fu) | (cand[pick[k + 1] * C::B + i] & 0xF0u));
+                } else {  // scale nibbles of choice groups 2q, 2q + 1
+                    const int k = 2 * (i - 74);
+                    v = static_cast<uint8_t>((cand[pick[k] * C::B + i] & 0x0Fu) | (cand[pick[k + 1] * C::B + i] & 0xF0u));
+                }
             } else if (FMT == IQ_FMT_IQ2_XS) {
                 if (i < 66) {
                     v = cand[pick[(i - 2) >> 2] * C::B + i];
@@ -421,7 +449,9 @@ __global__ void sqrt_diag_kernel(const float* hess, int64_t nblk, float* out) {
 
 cudaError_t launch_choice_search(int fmt, const ChoiceParams& p, int /*num_sms*/, cudaStream_t s) {
     if (p.rows == 0 || p.nblk == 0) return cudaSuccess;
-    return fmt == IQ_FMT_IQ1_S ? launch<IQ_FMT_IQ1_S>(p, s) : launch<IQ_FMT_IQ2_XS>(p, s);
+    if (fmt == IQ_FMT_IQ1_S) return launch<IQ_FMT_IQ1_S>(p, s);
+    if (fmt == IQ_FMT_IQ2_S) return launch<IQ_FMT_IQ2_S>(p, s);
+    return launch<IQ_FMT_IQ2_XS>(p, s);
 }
 
 cudaError_t launch_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t s) {

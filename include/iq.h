@@ -161,7 +161,7 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
 
 /*
  * Local-Hessian choice search (PR #3158 steps; one fused launch as in PR #3218) for the first
- * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S and IQ2_XS (other formats:
+ * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S, IQ2_XS and IQ2_S (IQ1_M:
  * IQ_EUNSUPPORTED).
  *   hess: fp32 [nblk][256][256], the symmetric diagonal block of the input Hessian per block,
  *     read as H[k][i] (row k, column i) for (H v)_i.

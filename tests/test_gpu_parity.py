@@ -29,7 +29,7 @@ def dev():
 @pytest.fixture(scope="module")
 def descs(dev, grids, anchors):
     out = {}
-    for fmt in ("iq1_s", "iq2_xs"):
+    for fmt in ("iq1_s", "iq2_xs", "iq2_s"):
         g = torch.from_numpy(grids[fmt]).to(dev)
         out[fmt] = iq.make_desc(fmt, g, anchors[fmt])
     return out
@@ -230,7 +230,7 @@ def _choice_case(fmt, rows, nblk, seed, offdiag):
     return w, hess
 
 
-@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s"])
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
 @pytest.mark.parametrize("offdiag", [0.02, 0.3])
 def test_choice_search_matches_oracle(dev, descs, grids, anchors, fmt, offdiag):
     rows, nblk = 13, 2
@@ -244,7 +244,7 @@ def test_choice_search_matches_oracle(dev, descs, grids, anchors, fmt, offdiag):
     assert np.array_equal(pay.cpu().numpy(), want_pay)
 
 
-@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s"])
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
 def test_local_hessian_pipeline_on_gpu_matches_oracle(dev, descs, grids, anchors, fmt):
     """sqrt(diag H) -> every-choice encode -> choice search, all in the library's kernels."""
     rows, nblk = 10, 3

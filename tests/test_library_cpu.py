@@ -94,6 +94,6 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert E(ctypes.byref(m), W, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
     assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 4
     s2 = _desc(fmt=4, entries=1024, anchor=0.9)
-    assert lib.iq_choice_search(ctypes.byref(s2), W, 4, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 4
+    assert lib.iq_choice_search(ctypes.byref(s2), W, 0, 1, 256, W, W, 1, 0, W, W, 1, None, None) == 2
     assert lib.iq_sqrt_diag(None, 1, W, None) == 1
     assert lib.iq_sqrt_diag(W, 0, W, None) == 2
