@@ -1,8 +1,8 @@
 """CPU oracle for the GGML IQ encoder path -- TEST INFRASTRUCTURE ONLY.
 
-A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS / IQ2_S encoder and decoder,
-and the local-Hessian choice search (IQ1_S, IQ2_XS), with this thin ctypes wrapper. It is the yardstick the CUDA library is
-checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS / IQ2_S encoder and
+decoder, and the local-Hessian choice search (IQ1_S, IQ2_XS, IQ2_S), with this thin ctypes wrapper.
+It is the yardstick the CUDA library is checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import it; the library never does, and the two share no code.
 
 Functions whose parity rests on invariants only (no value fixed by the pages or by a closed form)
@@ -57,7 +57,7 @@ def _load(path: str | None = None):
         lib.orc_decode.restype = None
         lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
         lib.orc_choice_search.restype = None
-        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, P, P, P, P]
+        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, i64, P, P, P, P]
         lib.orc_sqrt_diag.restype = None
         lib.orc_sqrt_diag.argtypes = [P, i64, P]
         lib.orc_f32_to_f16.restype = ctypes.c_uint16
@@ -162,24 +162,33 @@ def decode(fmt: str, grid: np.ndarray, payload: np.ndarray) -> np.ndarray:
 def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False):
     """Local-Hessian choice search over every 256-column block of w.
 
-    hess: [nblk, 256, 256] fp32; cand: [16, rows, nblk, B] every-choice payloads.
-    Returns (picks [rows, nblk, G], payload [rows, nblk, B]) and, with trace, the picks after
-    step 2 and after each sweep [rows, nblk, 3, G].
+    w: [rows, cols], or [experts, rows, cols] with hess [experts, nblk, 256, 256] (each expert's
+    rows use its own Hessian blocks); hess: [nblk, 256, 256] fp32 otherwise;
+    cand: [16, (experts,) rows, nblk, B] every-choice payloads.
+    Returns (picks [(experts,) rows, nblk, G], payload [(experts,) rows, nblk, B]) and, with
+    trace, the picks after step 2 and after each sweep [(experts,) rows, nblk, 3, G].
     Parity of the sweeps is pinned by the fp64 direct-objective replay in the tests.
     """
     wb = _bf16_bits(w)
-    rows, cols = wb.shape
+    lead = wb.shape[:-1]
+    cols = wb.shape[-1]
+    wb = wb.reshape(-1, cols)
+    rows = wb.shape[0]
+    nexp = wb.shape[0] // lead[-1] if len(lead) == 2 else 1
     nblk = cols // 256
     G, B = CHOICE_GROUPS[fmt], BLOCK_BYTES[fmt]
-    hess = np.ascontiguousarray(hess, dtype=np.float32).reshape(nblk, 256, 256)
+    hess = np.ascontiguousarray(hess, dtype=np.float32).reshape(nexp, nblk, 256, 256)
     cand = np.ascontiguousarray(cand, dtype=np.uint8).reshape(NUM_CHOICES, rows, nblk, B)
     picks = np.zeros((rows, nblk, G), dtype=np.uint8)
     payload = np.zeros((rows, nblk, B), dtype=np.uint8)
     tr = np.zeros((rows, nblk, 3, G), dtype=np.uint8) if trace else None
     _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
-                              rows, nblk, cols, _ptr(hess), _ptr(cand), _ptr(picks), _ptr(payload),
-                              _ptr(tr))
-    return (picks, payload, tr) if trace else (picks, payload)
+                              rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
+                              _ptr(payload), _ptr(tr))
+    picks, payload = picks.reshape(lead + (nblk, G)), payload.reshape(lead + (nblk, B))
+    if trace:
+        return picks, payload, tr.reshape(lead + (nblk, 3, G))
+    return picks, payload
 
 
 def sqrt_diag(hess: np.ndarray) -> np.ndarray:

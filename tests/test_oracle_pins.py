@@ -433,6 +433,34 @@ def test_choice_search_payload_is_the_encode_under_picks(grids, anchors, fmt):
     assert np.array_equal(payload, enc)
 
 
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s"])
+def test_choice_search_experts_use_their_own_hessians(grids, anchors, fmt):
+    """A stack of experts in one call equals one call per expert with that expert's H, and each
+    expert's decisions replay against its own H (the regime PR #3218 targets: many small
+    expert weights)."""
+    nexp, rows, nblk = 3, 3, 2
+    w = synth.normal_bf16((nexp, rows, nblk * 256), 0.02, 141)
+    hess = np.stack([np.stack([synth.block_hessian(150 + 10 * e + b, offdiag_std=0.3).numpy() for b in range(nblk)])
+                     for e in range(nexp)])                           # [E, nblk, 256, 256]
+    imp = oracle.sqrt_diag(hess).reshape(nexp, nblk * 256)
+    cand = np.stack([oracle.encode(fmt, grids[fmt], anchors[fmt], w[e], importance=imp[e], every_choice=True)[0]
+                     for e in range(nexp)], axis=1)                   # [16, E, rows, nblk, B]
+    picks, payload, trace = oracle.choice_search(fmt, grids[fmt], w, hess, cand, trace=True)
+    assert picks.shape[:3] == (nexp, rows, nblk)
+    G = oracle.CHOICE_GROUPS[fmt]
+    for e in range(nexp):
+        pe, ye = oracle.choice_search(fmt, grids[fmt], w[e], hess[e], cand[:, e])
+        assert np.array_equal(picks[e], pe) and np.array_equal(payload[e], ye)
+        for r in range(rows):
+            for b in range(nblk):
+                x = w[e].double().numpy()[r, 256 * b:256 * b + 256]
+                dl = x[None] - oracle.decode(fmt, grids[fmt], cand[:, e, r, b]).astype(np.float64)
+                viol, _, _ = replay_choice_search(dl, hess[e, b], G, trace[e, r, b], rel_tol=3e-5)
+                assert not viol, viol
+    other, _ = oracle.choice_search(fmt, grids[fmt], w, hess[[1, 2, 0]], cand)
+    assert not np.array_equal(other, picks)           # the Hessians do reach the decisions
+
+
 def test_sqrt_diag_matches_numpy():
     h = torch.stack([synth.block_hessian(7), synth.block_hessian(8)]).numpy()
     want = np.sqrt(np.stack([np.diag(h[0]), np.diag(h[1])]).astype(np.float32)).reshape(-1)
