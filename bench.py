@@ -200,6 +200,8 @@ class Workload:
             self._choice(synth.workload_choice_iq2xs(), "iq2_s")
         elif name == "choice_iq1s_4096x4096":
             self._choice(synth.workload_choice_iq2xs(), "iq1_s")
+        elif name == "choice_iq2xs_moe_16x1536x4096":
+            self._choice(synth.workload_choice_moe(), "iq2_xs")
         elif name == "iq1s_decode_1m_blocks":
             wl = synth.workload_iq1s_4096x4096_weighted()
             self._encode_decode(wl, "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 weighted payload x16)")
@@ -237,20 +239,23 @@ class Workload:
         self.fmt, self.kind = fmt, "choice"
         self.w_host, self.hess_host = wl["w"], wl["hess"]
         self.w, self.hess = wl["w"].to(self.dev), wl["hess"].to(self.dev)
-        rows, cols = self.w.shape
+        lead, cols = tuple(self.w.shape[:-1]), self.w.shape[-1]
         nblk = cols // 256
-        self.imp = torch.empty(cols, dtype=torch.float32, device=self.dev)
+        nexp = lead[0] if len(lead) == 2 else 1
+        self.imp = torch.empty((nexp, cols) if len(lead) == 2 else (cols,), dtype=torch.float32, device=self.dev)
         B, G = iq.BLOCK_BYTES[fmt], iq.CHOICE_GROUPS[fmt]
-        self.cand = torch.empty((16, rows, nblk, B), dtype=torch.uint8, device=self.dev)
-        self.picks = torch.empty((rows, nblk, G), dtype=torch.uint8, device=self.dev)
-        self.payload = torch.empty((rows, nblk, B), dtype=torch.uint8, device=self.dev)
+        self.cand = torch.empty((16,) + lead + (nblk, B), dtype=torch.uint8, device=self.dev)
+        self.picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=self.dev)
+        self.payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=self.dev)
         self.units = self.w.numel()
-        self.nblocks = rows * nblk
+        self.nblocks = self.units // 256
         self.launches_per_step = 3
+        shape = "x".join(str(v) for v in self.w.shape)
         self.text = (f"local-Hessian choice search, {fmt.upper()}: sqrt(diag H) + one-pass every-choice encode + "
-                     "two-sweep search, 4096x4096 bf16 N(0,0.02^2), 16 blocks of H = U^-1 U^-T")
+                     f"two-sweep search, {shape} bf16 N(0,0.02^2), one H = U^-1 U^-T per "
+                     + ("expert and " if nexp > 1 else "") + "256-column block")
         self.dominant = "choice_search_kernel"
-        self.ops_per_launch = rows * nblk * choice_ops_per_row_block(G)
+        self.ops_per_launch = self.nblocks * choice_ops_per_row_block(G)
         iq.iq_sqrt_diag(self.hess, out=self.imp)
         iq.iq_encode(self.desc[fmt], self.w, self.imp, every_choice=True, out=self.cand)
 
@@ -363,9 +368,13 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
     import oracle
     if name.startswith("choice_"):
         cfmt = {"choice_iq2xs_4096x4096": "iq2_xs", "choice_iq2s_4096x4096": "iq2_s",
-                "choice_iq1s_4096x4096": "iq1_s"}[name]
-        wl = synth.workload_choice_iq2xs()
-        w, hess = wl["w"], wl["hess"].numpy()
+                "choice_iq1s_4096x4096": "iq1_s", "choice_iq2xs_moe_16x1536x4096": "iq2_xs"}[name]
+        if "moe" in name:  # the sample is the first rows of expert 0, under its own Hessians
+            wl = synth.workload_choice_moe()
+            w, hess = wl["w"][0], wl["hess"][0].numpy()
+        else:
+            wl = synth.workload_choice_iq2xs()
+            w, hess = wl["w"], wl["hess"].numpy()
         g = {"iq2_xs": synth.iq2xs_grid, "iq2_s": synth.iq2s_grid, "iq1_s": synth.iq1s_grid}[cfmt]()
         imp = oracle.sqrt_diag(hess)
 

@@ -67,7 +67,7 @@ def load_library(path: str = LIB_PATH):
     lib.iq_decode.restype = ctypes.c_int
     lib.iq_decode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i32, P, P]
     lib.iq_choice_search.restype = ctypes.c_int
-    lib.iq_choice_search.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, P, i64, i64, P, P, i64, P, P]
+    lib.iq_choice_search.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, i64, P, i64, i64, P, P, i64, P, P]
     lib.iq_sqrt_diag.restype = ctypes.c_int
     lib.iq_sqrt_diag.argtypes = [P, i64, P, P]
     lib.iq_status_string.restype = ctypes.c_char_p
@@ -215,30 +215,41 @@ def iq_decode(desc: IQDesc, payload: torch.Tensor, out_dtype: torch.dtype = torc
 def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor,
                      picks: torch.Tensor | None = None, payload: torch.Tensor | None = None,
                      flags: torch.Tensor | None = None, stream=None):
-    """Local-Hessian choice search over all 256-column blocks of w [rows, cols].
+    """Local-Hessian choice search over all 256-column blocks of w.
 
-    hess: fp32 [cols/256, 256, 256]; cand: uint8 [16, rows, cols/256, B] (every-choice payloads).
-    Returns (picks uint8 [rows, cols/256, G], payload uint8 [rows, cols/256, B]).
+    w: bf16 [rows, cols] with hess fp32 [cols/256, 256, 256], or a stack of experts
+    [experts, rows, cols] with hess [experts, cols/256, 256, 256] (each expert's rows use its own
+    Hessian blocks; the experts must be contiguous in the row dimension).
+    cand: uint8 [16, (experts,) rows, cols/256, B], the every-choice payloads.
+    Returns (picks uint8 [(experts,) rows, cols/256, G], payload uint8 [(experts,) rows, cols/256, B]).
     """
     lib = load_library()
     fmt = _fmt_of(desc)
     _need(w, torch.bfloat16, "w")
     _need(hess, torch.float32, "hess")
     _need(cand, torch.uint8, "cand")
-    rows, cols = w.shape
+    if w.dim() not in (2, 3) or w.stride(-1) != 1:
+        raise IQError("w must be [rows, cols] or [experts, rows, cols] with a contiguous last dim")
+    lead, cols = tuple(w.shape[:-1]), w.shape[-1]
+    nexp, rows_e = (lead[0], lead[1]) if w.dim() == 3 else (1, lead[0])
+    if w.dim() == 3 and nexp > 1 and w.stride(0) != rows_e * w.stride(1):
+        raise IQError("the experts of w must be contiguous in the row dimension")
+    rows = nexp * rows_e
     nblk = cols // 256
     B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
-    if w.stride(-1) != 1 or not hess.is_contiguous() or hess.numel() != nblk * 256 * 256:
-        raise IQError("w needs a contiguous last dim; hess must be contiguous [cols/256, 256, 256]")
-    if tuple(cand.shape) != (NUM_CHOICES, rows, nblk, B) or not cand.is_contiguous():
-        raise IQError(f"cand must be contiguous {(NUM_CHOICES, rows, nblk, B)}")
+    if not hess.is_contiguous() or hess.numel() != nexp * nblk * 256 * 256:
+        raise IQError("hess must be contiguous [(experts,) cols/256, 256, 256]")
+    want = (NUM_CHOICES,) + lead + (nblk, B)
+    if tuple(cand.shape) != want or not cand.is_contiguous():
+        raise IQError(f"cand must be contiguous {want}")
     if picks is None:
-        picks = torch.empty((rows, nblk, G), dtype=torch.uint8, device=w.device)
+        picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=w.device)
     if payload is None:
-        payload = torch.empty((rows, nblk, B), dtype=torch.uint8, device=w.device)
-    _check(lib.iq_choice_search(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(0), hess.data_ptr(),
-                                cand.data_ptr(), nblk, rows * nblk * B, picks.data_ptr(), payload.data_ptr(),
-                                nblk, None if flags is None else flags.data_ptr(), _stream(stream)))
+        payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=w.device)
+    _check(lib.iq_choice_search(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(-2), hess.data_ptr(),
+                                rows_e, cand.data_ptr(), nblk, rows * nblk * B, picks.data_ptr(),
+                                payload.data_ptr(), nblk, None if flags is None else flags.data_ptr(),
+                                _stream(stream)))
     return picks, payload
 
 

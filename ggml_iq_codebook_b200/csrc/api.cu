@@ -133,7 +133,7 @@ iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks
 }
 
 iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows, int64_t nblk,
-                           int64_t ldw, const float* hess, const uint8_t* cand, int64_t cand_ld,
+                           int64_t ldw, const float* hess, int64_t rows_per_hess, const uint8_t* cand, int64_t cand_ld,
                            int64_t cand_choice_stride, uint8_t* picks, uint8_t* payload,
                            int64_t payload_ld, uint32_t* flags, cudaStream_t stream) {
     iq_status st = check_desc(desc);
@@ -144,6 +144,8 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;
     if (ldw < nblk * 256 || ldw % 8 != 0 || !aligned(w, 16) || !aligned(hess, 16)) return IQ_EINVAL;
     if (cand_ld < nblk || payload_ld < nblk || cand_choice_stride < 0) return IQ_EINVAL;
+    if (rows_per_hess == 0) rows_per_hess = rows;
+    if (rows_per_hess < 0 || rows % rows_per_hess != 0) return IQ_ESHAPE;
     int sms = 0;
     if ((st = device_sms(&sms)) != IQ_OK) return st;
     if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
@@ -153,6 +155,7 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     p.nblk = nblk;
     p.ldw = ldw;
     p.hess = hess;
+    p.rows_per_hess = rows_per_hess;
     p.cand = cand;
     p.cand_ld = cand_ld;
     p.cand_cstride = cand_choice_stride;

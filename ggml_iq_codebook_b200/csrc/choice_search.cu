@@ -15,6 +15,9 @@
 //
 // Formats: IQ1_S (8 groups of 32 columns), IQ2_XS and IQ2_S (16 groups of 16 columns); 16 choices.
 //
+// Experts: a stack of weights sharing a row layout runs in the same launch, row r taking Hessian
+// set r / rows_per_hess (PR #3218's reason for one launch: thousands of small expert weights).
+//
 // Design (B200): one CTA = 16 (IQ2_XS, IQ2_S) or 8 (IQ1_S) rows of one block, a half-warp per row and
 // one lane per choice. The
 // rows run the group steps in lockstep, so each step stages one panel of H (the group's W rows,
@@ -197,20 +200,25 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     int* swf = reinterpret_cast<int*>(smem + C::oSw);
     uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem + C::oGrid);
 
-    const int64_t row_tiles = (p.rows + kRows - 1) / kRows;
-    const int64_t blk = blockIdx.x / row_tiles;
-    const int64_t row0 = (blockIdx.x - blk * row_tiles) * kRows;
+    // CTA -> (block, expert, row tile): a tile never straddles two experts, and the CTAs that
+    // share one Hessian block are adjacent in launch order.
+    const int64_t nexp = p.rows / p.rows_per_hess;
+    const int64_t tiles_e = (p.rows_per_hess + kRows - 1) / kRows;
+    const int64_t blk = blockIdx.x / (nexp * tiles_e);
+    const int64_t rem = blockIdx.x - blk * nexp * tiles_e;
+    const int64_t expert = rem / tiles_e;
+    const int64_t tile_row0 = (rem - expert * tiles_e) * kRows;
     const int tid = threadIdx.x, hr = tid >> 4, c = tid & 15;
     const unsigned hmask = 0xFFFFu << (16 * (hr & 1));  // this half-warp's lanes within the warp
-    const int64_t row = row0 + hr;
-    const bool active = row < p.rows;
+    const int64_t row = expert * p.rows_per_hess + tile_row0 + hr;
+    const bool active = tile_row0 + hr < p.rows_per_hess;
     char* rec = smem + C::oRows + hr * C::rBytes;
     uint16_t* xb = reinterpret_cast<uint16_t*>(rec + C::rX);
     float* cur = reinterpret_cast<float*>(rec + C::rCur);
     float* grad = reinterpret_cast<float*>(rec + C::rGrad);
     int* pick = reinterpret_cast<int*>(rec + C::rPick);
     uint8_t* cand = reinterpret_cast<uint8_t*>(rec + C::rCand);
-    const float* H = p.hess + blk * kBlock * kBlock;
+    const float* H = p.hess + (expert * p.nblk + blk) * kBlock * kBlock;
 
     // H panels (the W rows of one choice group) stream through a double buffer: step s of the
     // 3G group steps (step 2, then two sweeps) uses panel s % G from buffer s & 1.
@@ -433,7 +441,7 @@ cudaError_t launch(const ChoiceParams& p, cudaStream_t s) {
     auto kern = choice_search_kernel<FMT>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem);
     if (err != cudaSuccess) return err;
-    const int64_t ctas = p.nblk * ((p.rows + C::R - 1) / C::R);
+    const int64_t ctas = p.nblk * (p.rows / p.rows_per_hess) * ((p.rows_per_hess + C::R - 1) / C::R);
     kern<<<static_cast<unsigned>(ctas), C::T, C::smem, s>>>(p);
     return cudaGetLastError();
 }

@@ -34,6 +34,7 @@ struct ChoiceParams {
     const uint16_t* w;
     int64_t rows, nblk, ldw;
     const float* hess;
+    int64_t rows_per_hess;  // row r uses Hessian set r / rows_per_hess (divides rows)
     const uint8_t* cand;
     int64_t cand_ld, cand_cstride;
     uint8_t* picks;

@@ -153,3 +153,12 @@ def workload_choice_iq2xs(device="cpu", rows=4096, cols=4096):
     nblk = cols // BLOCK
     hess = torch.stack([block_hessian(5000 + b) for b in range(nblk)]).to(device)
     return {"fmt": "iq2_xs", "w": normal_bf16((rows, cols), 0.02, 1005, device), "hess": hess}
+
+
+def workload_choice_moe(device="cpu", experts=16, rows=1536, cols=4096):
+    """Local-Hessian choice search over a stack of expert weights [experts, rows, cols], N(0, 0.02^2),
+    each expert with its own H per 256-column block ([experts, nblk, 256, 256])."""
+    nblk = cols // BLOCK
+    hess = torch.stack([torch.stack([block_hessian(6000 + nblk * e + b) for b in range(nblk)])
+                        for e in range(experts)]).to(device)
+    return {"fmt": "iq2_xs", "w": normal_bf16((experts, rows, cols), 0.02, 1006, device), "hess": hess}

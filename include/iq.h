@@ -163,8 +163,11 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
  * Local-Hessian choice search (PR #3158 steps; one fused launch as in PR #3218) for the first
  * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S, IQ2_XS and IQ2_S (IQ1_M:
  * IQ_EUNSUPPORTED).
- *   hess: fp32 [nblk][256][256], the symmetric diagonal block of the input Hessian per block,
- *     read as H[k][i] (row k, column i) for (H v)_i.
+ *   hess: fp32 [rows / rows_per_hess][nblk][256][256], the symmetric diagonal blocks of the input
+ *     Hessian, read as H[k][i] (row k, column i) for (H v)_i. Row r uses set r / rows_per_hess:
+ *     a stack of experts that share a row layout runs in one call, each with its own Hessian
+ *     (PR #3218: launch overhead dominated on MoE models). rows_per_hess = 0 means rows (one set);
+ *     otherwise it must divide rows (IQ_ESHAPE).
  *   cand: the every-choice payloads of those blocks; candidate c of (row r, block b) starts at
  *     cand + c * cand_choice_stride + (r * cand_ld + b) * B   (bytes; cand_ld in blocks).
  *   picks: uint8 [rows][nblk][G], the chosen choice of every choice group.
@@ -177,8 +180,8 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
  * then grad += H[:, g] u. Lowest choice on equal score or gain.
  */
 iq_status iq_choice_search(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t nblk,
-                           int64_t ldw, const float *hess, const uint8_t *cand, int64_t cand_ld,
-                           int64_t cand_choice_stride, uint8_t *picks, uint8_t *payload,
+                           int64_t ldw, const float *hess, int64_t rows_per_hess, const uint8_t *cand,
+                           int64_t cand_ld, int64_t cand_choice_stride, uint8_t *picks, uint8_t *payload,
                            int64_t payload_ld, uint32_t *flags, cudaStream_t stream);
 
 /*

@@ -265,6 +265,31 @@ def test_local_hessian_pipeline_on_gpu_matches_oracle(dev, descs, grids, anchors
     assert torch.equal(fixed, pay)
 
 
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
+def test_choice_search_over_a_stack_of_experts(dev, descs, grids, anchors, fmt):
+    """Experts of 13 rows (ragged against the 16- and 8-row CTA tiles), each with its own
+    Hessian blocks, in one batched encode and one choice-search launch."""
+    nexp, rows, nblk = 3, 13, 2
+    w = synth.normal_bf16((nexp, rows, nblk * 256), 0.02, 521)
+    hess = torch.stack([torch.stack([synth.block_hessian(530 + 10 * e + b, offdiag_std=0.3) for b in range(nblk)])
+                        for e in range(nexp)])                        # [E, nblk, 256, 256]
+    hd = hess.to(dev)
+    imp_d = iq.iq_sqrt_diag(hd).view(nexp, nblk * 256)
+    cand_d = iq.iq_encode(descs[fmt], w.to(dev), imp_d, every_choice=True)   # [16, E, rows, nblk, B]
+    picks, pay = iq.iq_choice_search(descs[fmt], w.to(dev), hd, cand_d)
+    torch.cuda.synchronize()
+    imp = oracle.sqrt_diag(hess.numpy()).reshape(nexp, nblk * 256)
+    cand = np.stack([oracle.encode(fmt, grids[fmt], anchors[fmt], w[e], importance=imp[e], every_choice=True)[0]
+                     for e in range(nexp)], axis=1)
+    assert np.array_equal(cand_d.cpu().numpy(), cand)
+    want_p, want_pay = oracle.choice_search(fmt, grids[fmt], w, hess.numpy(), cand)
+    assert np.array_equal(picks.cpu().numpy(), want_p)
+    assert np.array_equal(pay.cpu().numpy(), want_pay)
+    for e in range(nexp):                             # and the same as one launch per expert
+        pe, ye = iq.iq_choice_search(descs[fmt], w[e].to(dev), hd[e].contiguous(), cand_d[:, e].contiguous())
+        assert torch.equal(pe, picks[e]) and torch.equal(ye, pay[e])
+
+
 # --------------------------------------------------------------------------------- full sizes
 
 def _sample_rows(rows, k, seed):
