@@ -144,6 +144,7 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;
     if (ldw < nblk * 256 || ldw % 8 != 0 || !aligned(w, 16) || !aligned(hess, 16)) return IQ_EINVAL;
     if (cand_ld < nblk || payload_ld < nblk || cand_choice_stride < 0) return IQ_EINVAL;
+    if (!aligned(cand, 2) || (cand_choice_stride & 1) != 0) return IQ_EINVAL;  // 2-byte staging
     if (rows_per_hess == 0) rows_per_hess = rows;
     if (rows_per_hess < 0 || rows % rows_per_hess != 0) return IQ_ESHAPE;
     int sms = 0;

@@ -28,8 +28,10 @@
 // by broadcast 16-byte panel reads. Its two trees are local, and the only cross-lane step is a
 // 4-level argmin over the half-warp; the winning lane writes cur and u from its registers. The
 // gradient work (the initial H Delta, and after every sweep step the updates of the rows that
-// switched) is done by all threads together as 4-row x 4-column register tiles: per k one 16-byte
-// read of the rows' values and one of H, then 16 fmas. The grid is staged as
+// switched) is done by all threads together: the initial H Delta as 4-row x 4-column register
+// tiles (per k one 16-byte read of the rows' values and one of H, then 16 fmas); after a sweep
+// step, by column when few rows switched (each thread holding its H column and walking only those
+// rows), else by the same tiles. The grid is staged as
 // 16-bit element codes, so decoding needs no int-to-float conversions.
 #include "iq_device.cuh"
 #include "iq_kernels.h"
@@ -60,6 +62,12 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
     return static_cast<uint16_t>(c);
 }
 
+// float(n) for 0 <= n < 2^23, exactly, without an int-to-float conversion (those throttle the
+// MIO queue): the bits 2^23 + n, minus 2^23.
+__device__ __forceinline__ float small_int_to_float(uint32_t n) {
+    return __fsub_rn(__uint_as_float(0x4B000000u | n), 8388608.0f);
+}
+
 // The decoded values of one 8-weight group of candidate `pc`: xh[j] = value of element j of
 // 8-weight group `grp8` (inside the block) in choice group g. The products the group can take are
 // formed once (IQ1_S: s (q + delta), q in {-1, 0, 1}; IQ2_XS: s g, g in {1, 3, 5, 7}), each
@@ -72,7 +80,7 @@ __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid
         // shift 2 (grp8 % 4) of byte 66 + grp8 / 4, choice group g's scale nibble at 74 + g / 2
         const uint32_t sc = pc[74 + (g >> 1)];
         const int ls = static_cast<int>((g & 1) ? (sc >> 4) : (sc & 15u));
-        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float s = __fmul_rn(d, small_int_to_float(static_cast<uint32_t>(2 * ls + 1)));
         const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
         const uint32_t idx = static_cast<uint32_t>(pc[2 + grp8]) | (((static_cast<uint32_t>(pc[66 + (grp8 >> 2)]) >> (2 * (grp8 & 3))) & 3u) << 8);
         const uint32_t neg = pc[34 + grp8];
@@ -87,7 +95,7 @@ __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid
         const uint32_t code = *reinterpret_cast<const uint16_t*>(pc + 2 + 2 * grp8);
         const uint32_t sc = pc[66 + (g >> 1)];
         const int ls = static_cast<int>((g & 1) ? (sc >> 4) : (sc & 15u));
-        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float s = __fmul_rn(d, small_int_to_float(static_cast<uint32_t>(2 * ls + 1)));
         const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
         const uint32_t sign7 = code >> 9;
         const uint32_t neg = sign7 | (static_cast<uint32_t>(__popc(sign7) & 1) << 7);
@@ -100,7 +108,7 @@ __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid
         }
     } else {
         const uint32_t qh = *reinterpret_cast<const uint16_t*>(pc + 34 + 2 * g);
-        const float s = __fmul_rn(d, static_cast<float>(2 * static_cast<int>((qh >> 12) & 7u) + 1));
+        const float s = __fmul_rn(d, small_int_to_float(2u * ((qh >> 12) & 7u) + 1u));
         const float delta = (qh & 0x8000u) ? -0.125f : 0.125f;
         const float vp = __fmul_rn(s, __fadd_rn(1.0f, delta));
         const float v0 = __fmul_rn(s, __fadd_rn(0.0f, delta));
@@ -121,6 +129,13 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 
+#ifndef IQ_CHOICE_COLUMN_MAX_W16
+#define IQ_CHOICE_COLUMN_MAX_W16 12  // 16-column choice groups (IQ2_XS, IQ2_S), 16 rows per CTA
+#endif
+#ifndef IQ_CHOICE_COLUMN_MAX_W32
+#define IQ_CHOICE_COLUMN_MAX_W32 0  // 32-column choice groups (IQ1_S): always tiles (measured)
+#endif
+
 template <int FMT>
 struct Cfg {
     static constexpr int R = FMT == IQ_FMT_IQ1_S ? 8 : 16;      // rows per CTA (shared-memory budget)
@@ -133,9 +148,13 @@ struct Cfg {
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
     // shared memory layout (bytes)
     static constexpr int oHp = 0;                                 // float [2][W][256], double buffer
-    static constexpr int oCurT = oHp + 2 * W * kBlock * 4;        // float [256][R]
-    static constexpr int oUT = oCurT + kBlock * R * 4;            // float [W][R]: the switches' u
-    static constexpr int oSw = oUT + W * R * 4;                   // int [R]: row switched this step
+    static constexpr int oCurT = oHp + 2 * W * kBlock * 4;        // float [256][R], step 2 only
+    // the sweeps' u of the rows that switched, in the curT area (free once step 2 is done)
+    static constexpr int oUT = oCurT;                             // float [W][R]
+    static constexpr int oUR = oUT + W * R * 4;                   // float [R][W]: the same, by row
+    static constexpr int oSw = oCurT + kBlock * R * 4;            // int [R]: row switched this step
+    // update by column up to this many switched rows, else by tiles (either is bit-exact)
+    static constexpr int COLUMN_MAX = W == 16 ? IQ_CHOICE_COLUMN_MAX_W16 : IQ_CHOICE_COLUMN_MAX_W32;
     static constexpr int oGrid = oSw + R * 4;                     // uint16 [E] element codes
     static constexpr int oRows = oGrid + (E * 2 + 15) / 16 * 16;  // per-row records
     static constexpr int rX = 0;                                  // bf16 [256]
@@ -194,9 +213,11 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     using C = Cfg<FMT>;
     constexpr int W = C::W, G = C::G, kRows = C::R, kThreads = C::T;
     static_assert(kThreads == C::RG * 64, "gradient tiles: 4 rows x 4 columns per thread");
+    static_assert(2 * W * kRows <= kBlock * kRows, "u buffers fit in the curT area");
     extern __shared__ __align__(16) char smem[];
     float* curT = reinterpret_cast<float*>(smem + C::oCurT);
     float* uT = reinterpret_cast<float*>(smem + C::oUT);
+    float* uR = reinterpret_cast<float*>(smem + C::oUR);
     int* swf = reinterpret_cast<int*>(smem + C::oSw);
     uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem + C::oGrid);
 
@@ -246,8 +267,15 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
             for (int j = 0; j < 8; ++j) nonfinite |= !isfinite(xv[j]);
         }
         if (__any_sync(hmask, nonfinite) && c == 0) raise_flags(p.flags, IQ_FLAG_NONFINITE);
-        const uint8_t* src = p.cand + c * p.cand_cstride + (row * p.cand_ld + blk) * C::B;
-        for (int i = 0; i < C::B; ++i) cand[c * C::B + i] = src[i];
+        // 2-byte copies (B is even and the caller's candidates are 2-byte aligned), all loads
+        // issued before the stores
+        const uint16_t* src = reinterpret_cast<const uint16_t*>(p.cand + c * p.cand_cstride + (row * p.cand_ld + blk) * C::B);
+        uint16_t* dst = reinterpret_cast<uint16_t*>(cand + c * C::B);
+        uint16_t stage[C::B / 2];
+#pragma unroll
+        for (int i = 0; i < C::B / 2; ++i) stage[i] = __ldg(src + i);
+#pragma unroll
+        for (int i = 0; i < C::B / 2; ++i) dst[i] = stage[i];
     } else {
         for (int i = c; i < kBlock; i += 16) curT[i * kRows + hr] = 0.0f;
     }
@@ -367,15 +395,40 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
                 for (int i = 0; i < W; ++i) uT[i * kRows + hr] = u[i];
 #pragma unroll
                 for (int i = 0; i < W; i += 4)
+                    *reinterpret_cast<float4*>(uR + hr * W + i) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
+#pragma unroll
+                for (int i = 0; i < W; i += 4)
                     *reinterpret_cast<float4*>(cur + g * W + i) = make_float4(dl[i], dl[i + 1], dl[i + 2], dl[i + 3]);
                 pick[g] = c;
             }
         }
         if (c == 0) swf[hr] = switched;
         __syncthreads();
-        // grad[r][i] += sum_k H[k][i] u_k (fma chain over the group's k) for the switched rows
-        const bool any4 = swf[4 * rg] | swf[4 * rg + 1] | swf[4 * rg + 2] | swf[4 * rg + 3];
-        if (any4) {
+        // grad[r][i] += sum_k H[k][i] u_k (fma chain over the group's k, the same order either
+        // way) for the rows that switched. Few switches: by column, each thread holding H[k][i]
+        // for its columns in registers and walking only those rows. Many: 4-row x 4-column
+        // register tiles over every 4-row group with a switch, writing back only switched rows.
+        uint32_t swmask = 0;
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) swmask |= static_cast<uint32_t>(swf[r] != 0) << r;
+        if (swmask != 0 && __popc(swmask) <= C::COLUMN_MAX) {
+#pragma unroll
+            for (int i = tid; i < kBlock; i += kThreads) {
+                float hcol[W];
+#pragma unroll
+                for (int k = 0; k < W; ++k) hcol[k] = Hp[k * kBlock + i];
+                for (uint32_t m = swmask; m != 0; m &= m - 1) {
+                    const int r = __ffs(m) - 1;
+                    float uk[W];
+                    load_vec<W>(uR + r * W, uk);
+                    float* gr = grad_row(r);
+                    float acc = gr[i];
+#pragma unroll
+                    for (int k = 0; k < W; ++k) acc = __fmaf_rn(hcol[k], uk[k], acc);
+                    gr[i] = acc;
+                }
+            }
+        } else if (swmask != 0 && ((swmask >> (4 * rg)) & 15u) != 0) {
             float acc[4][4];
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
@@ -394,7 +447,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
             }
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr)
-                if (swf[4 * rg + rr])  // rows that kept their choice keep their gradient bit for bit
+                if ((swmask >> (4 * rg + rr)) & 1u)  // rows that kept their choice keep their gradient
                     *reinterpret_cast<float4*>(grad_row(4 * rg + rr) + 4 * cg) =
                         make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
         }

@@ -169,7 +169,8 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
  *     (PR #3218: launch overhead dominated on MoE models). rows_per_hess = 0 means rows (one set);
  *     otherwise it must divide rows (IQ_ESHAPE).
  *   cand: the every-choice payloads of those blocks; candidate c of (row r, block b) starts at
- *     cand + c * cand_choice_stride + (r * cand_ld + b) * B   (bytes; cand_ld in blocks).
+ *     cand + c * cand_choice_stride + (r * cand_ld + b) * B   (bytes; cand_ld in blocks). cand is
+ *     2-byte aligned and cand_choice_stride even (IQ_EINVAL otherwise).
  *   picks: uint8 [rows][nblk][G], the chosen choice of every choice group.
  *   payload: the final payload, block (r, b) at payload + (r * payload_ld + b) * B: each choice
  *     group's fields copied from its picked candidate, d from candidate 0 (the encode under the
