@@ -62,12 +62,6 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
     return static_cast<uint16_t>(c);
 }
 
-// float(n) for 0 <= n < 2^23, exactly, without an int-to-float conversion (those throttle the
-// MIO queue): the bits 2^23 + n, minus 2^23.
-__device__ __forceinline__ float small_int_to_float(uint32_t n) {
-    return __fsub_rn(__uint_as_float(0x4B000000u | n), 8388608.0f);
-}
-
 // The decoded values of one 8-weight group of candidate `pc`: xh[j] = value of element j of
 // 8-weight group `grp8` (inside the block) in choice group g. The products the group can take are
 // formed once (IQ1_S: s (q + delta), q in {-1, 0, 1}; IQ2_XS: s g, g in {1, 3, 5, 7}), each

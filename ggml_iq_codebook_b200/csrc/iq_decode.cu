@@ -95,7 +95,7 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
         const uint32_t w0 = pw[24], w1 = pw[25], w2 = pw[26], w3 = pw[27];
         const float d = half_bits_to_f32(iq1m_d_bits(w0, w1, w2, w3));
         const uint32_t wk = pw[24 + (h >> 2)];
-        const float s = __fmul_rn(d, static_cast<float>(2 * static_cast<int>((wk >> (3 * (h & 3))) & 7u) + 1));
+        const float s = __fmul_rn(d, small_int_to_float(2u * ((wk >> (3 * (h & 3))) & 7u) + 1u));
         const uint32_t lw = pw[h];      // low index bytes of groups 2h, 2h + 1
         const uint32_t nb = pb[32 + h];  // their nibbles
 #pragma unroll
@@ -117,7 +117,7 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
     if (FMT == IQ_FMT_IQ2_S) {
         const uint32_t sc = pb[74 + (h >> 1)];
         const int ls = static_cast<int>((h & 1) ? (sc >> 4) : (sc & 15u));
-        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float s = __fmul_rn(d, small_int_to_float(static_cast<uint32_t>(2 * ls + 1)));
         const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
         const uint32_t lw = pw[1 + h];                  // low index bytes of groups 2h, 2h + 1
         const uint32_t sg = pw[17 + h];                 // their sign bytes
@@ -140,7 +140,7 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
     if (FMT == IQ_FMT_IQ1_S) {
         const uint32_t lw = pw[1 + h];          // low index bytes of groups 2h, 2h + 1
         const uint32_t qh = pw[17 + (h >> 1)];  // the sub-block's qh
-        const float s = __fmul_rn(d, static_cast<float>(2 * static_cast<int>((qh >> 12) & 7u) + 1));
+        const float s = __fmul_rn(d, small_int_to_float(2u * ((qh >> 12) & 7u) + 1u));
         const float delta = (qh & 0x8000u) ? -0.125f : 0.125f;
         const float vp = __fmul_rn(s, __fadd_rn(1.0f, delta));   // q = +1
         const float v0 = __fmul_rn(s, __fadd_rn(0.0f, delta));   // q = 0
@@ -157,7 +157,7 @@ __device__ __forceinline__ void decode_pair(const uint8_t* pb, int h, const uint
         const uint32_t ca = pw[1 + 2 * h], cb = pw[2 + 2 * h];  // codes of groups 2h, 2h + 1
         const uint32_t sc = pb[66 + (h >> 1)];                   // scales of sub-blocks 2(h/2), +1
         const int ls = static_cast<int>((h & 1) ? (sc >> 4) : (sc & 15u));
-        const float s = __fmul_rn(d, static_cast<float>(2 * ls + 1));
+        const float s = __fmul_rn(d, small_int_to_float(static_cast<uint32_t>(2 * ls + 1)));
         const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
