@@ -53,7 +53,8 @@ def _load(path: str | None = None):
         P = ctypes.c_void_p
         i64 = ctypes.c_int64
         lib.orc_encode.restype = ctypes.c_uint32
-        lib.orc_encode.argtypes = [ctypes.c_int, P, ctypes.c_float, P, i64, i64, P, P, ctypes.c_int, P, P]
+        lib.orc_encode.argtypes = [ctypes.c_int, P, ctypes.c_float, P, ctypes.c_int, i64, i64, P, P, ctypes.c_int,
+                                   P, P]
         lib.orc_decode.restype = None
         lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
         lib.orc_choice_search.restype = None
@@ -97,6 +98,30 @@ def _bf16_bits(w) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(w, dtype=np.uint16))
 
 
+IN_BF16, IN_F16, IN_F32 = 0, 1, 2
+
+
+def _weights(w):
+    """(contiguous array, element kind) for a torch bf16/f16/f32 tensor, a numpy float32/float16
+    array, or a uint16 array of bf16 bit patterns."""
+    if hasattr(w, "dtype") and str(w.dtype).startswith("torch."):
+        import torch
+        t = w.detach().cpu().contiguous()
+        if t.dtype == torch.bfloat16:
+            return np.ascontiguousarray(t.view(torch.int16).numpy().view(np.uint16)), IN_BF16
+        if t.dtype == torch.float16:
+            return np.ascontiguousarray(t.view(torch.int16).numpy().view(np.uint16)), IN_F16
+        if t.dtype == torch.float32:
+            return np.ascontiguousarray(t.numpy()), IN_F32
+        raise TypeError(f"unsupported weight dtype {t.dtype}")
+    a = np.asarray(w)
+    if a.dtype == np.float32:
+        return np.ascontiguousarray(a), IN_F32
+    if a.dtype == np.float16:
+        return np.ascontiguousarray(a.view(np.uint16)), IN_F16
+    return np.ascontiguousarray(a.astype(np.uint16)), IN_BF16
+
+
 def set_threads(n: int) -> None:
     _load().orc_set_threads(int(n))
 
@@ -122,14 +147,14 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
 
 def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choices=None,
            every_choice: bool = False, scales=None):
-    """Encode a [rows, cols] bf16 weight. Returns (payload uint8, flags).
+    """Encode a [rows, cols] weight (bf16, f16 or f32; see _weights). Returns (payload uint8, flags).
 
     payload: [rows, cols/256, B], or [C, rows, cols/256, B] with every_choice (C = 16; 8 for iq1_m).
     anchor is ignored for iq1_m, whose anchor follows each block's peak-to-RMS.
     scales: optional [rows, cols/256] fp16 values (or their uint16 bits): encode under these d.
     """
     lib = _load()
-    wb = _bf16_bits(w)
+    wb, kind = _weights(w)
     rows, cols = wb.shape
     if cols % 256:
         raise ValueError("cols must be a multiple of 256")
@@ -144,7 +169,7 @@ def encode(fmt: str, grid: np.ndarray, anchor: float, w, importance=None, choice
         sc = np.ascontiguousarray(sc.view(np.uint16) if sc.dtype == np.float16 else sc.astype(np.uint16))
     shape = (CHOICES[fmt], rows, nblk, B) if every_choice else (rows, nblk, B)
     out = np.zeros(shape, dtype=np.uint8)
-    flags = lib.orc_encode(FMT[fmt], _ptr(grid), float(anchor), _ptr(wb), rows, cols, _ptr(imp),
+    flags = lib.orc_encode(FMT[fmt], _ptr(grid), float(anchor), _ptr(wb), kind, rows, cols, _ptr(imp),
                            _ptr(ch), int(bool(every_choice)), _ptr(sc), _ptr(out))
     return out, int(flags)
 
