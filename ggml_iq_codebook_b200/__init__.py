@@ -29,6 +29,7 @@ NUM_CHOICES = 16
 DEFAULT_ANCHOR = {"iq1_s": 0.61, "iq2_xs": 0.9, "iq1_m": 1.0, "iq2_s": 0.9}
 
 IQ_OUT_F32, IQ_OUT_BF16 = 0, 1
+IQ_IN = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
 
 SYMBOLS = ("iq_block_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
@@ -63,7 +64,8 @@ def load_library(path: str = LIB_PATH):
     lib.iq_num_choices.restype = i32
     lib.iq_num_choices.argtypes = [i32]
     lib.iq_encode.restype = ctypes.c_int
-    lib.iq_encode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, i64, i64, P, i64, P, P, i64, i32, P, P, P]
+    lib.iq_encode.argtypes = [ctypes.POINTER(IQDesc), P, i32, i64, i64, i64, i64, i64, P, i64, P, P, i64, i32, P, P,
+                              P]
     lib.iq_decode.restype = ctypes.c_int
     lib.iq_decode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i32, P, P]
     lib.iq_choice_search.restype = ctypes.c_int
@@ -113,7 +115,7 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
               choices: torch.Tensor | None = None, every_choice: bool = False,
               out: torch.Tensor | None = None, flags: torch.Tensor | None = None, stream=None,
               raise_on_flags: bool = True, scales: torch.Tensor | None = None) -> torch.Tensor:
-    """Encode bf16 weights [rows, cols] or [batch, rows, cols] (last dim contiguous).
+    """Encode weights [rows, cols] or [batch, rows, cols] (bf16, f16 or f32; last dim contiguous).
 
     importance: fp32 [cols] or [batch, cols]; choices: uint8 [..., rows, cols/256, G].
     scales: static block scales, either fp16 [..., rows, cols/256] (contiguous) or, except for
@@ -125,7 +127,8 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
     """
     lib = load_library()
     fmt = _fmt_of(desc)
-    _need(w, torch.bfloat16, "w")
+    if not isinstance(w, torch.Tensor) or not w.is_cuda or w.dtype not in IQ_IN:
+        raise IQError("w must be a CUDA tensor of bfloat16, float16 or float32")
     batched = w.dim() == 3
     if w.dim() not in (2, 3) or w.stride(-1) != 1:
         raise IQError("w must be [rows, cols] or [batch, rows, cols] with a contiguous last dim")
@@ -169,7 +172,7 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
     if flags is None:
         flags = torch.empty(1, dtype=torch.int32, device=w.device)
     flags_ptr = None if flags is False else flags.data_ptr()
-    _check(lib.iq_encode(ctypes.byref(desc), w.data_ptr(), batch, rows, cols, ldw, wbs, imp_ptr, imp_bs,
+    _check(lib.iq_encode(ctypes.byref(desc), w.data_ptr(), IQ_IN[w.dtype], batch, rows, cols, ldw, wbs, imp_ptr, imp_bs,
                          ch_ptr, sc_ptr, sc_stride, int(bool(every_choice)), out.data_ptr(), flags_ptr,
                          _stream(stream)))
     if raise_on_flags and flags is not False:

@@ -70,7 +70,7 @@ int32_t iq_num_choices(int32_t fmt) {
     return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS || fmt == IQ_FMT_IQ2_S) ? 16 : fmt == IQ_FMT_IQ1_M ? 8 : 0;
 }
 
-iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64_t rows, int64_t cols,
+iq_status iq_encode(const iq_desc* desc, const void* w, int32_t w_dtype, int64_t batch, int64_t rows, int64_t cols,
                     int64_t ldw, int64_t w_batch_stride, const float* importance,
                     int64_t imp_batch_stride, const uint8_t* choices, const uint16_t* scales,
                     int64_t scales_stride, int32_t every_choice, uint8_t* payload, uint32_t* flags, cudaStream_t stream) {
@@ -78,8 +78,10 @@ iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64
     if (st != IQ_OK) return st;
     if (w == nullptr || payload == nullptr) return IQ_EINVAL;
     if (batch <= 0 || rows <= 0 || cols <= 0 || cols % 256 != 0) return IQ_ESHAPE;
-    if (ldw < cols || ldw % 8 != 0 || !aligned(w, 16)) return IQ_EINVAL;
-    if (batch > 1 && (w_batch_stride < (rows - 1) * ldw + cols || w_batch_stride % 8 != 0)) return IQ_EINVAL;
+    if (w_dtype != IQ_IN_BF16 && w_dtype != IQ_IN_F16 && w_dtype != IQ_IN_F32) return IQ_EINVAL;
+    const int64_t vec = w_dtype == IQ_IN_F32 ? 4 : 8;  // elements per 16 bytes
+    if (ldw < cols || ldw % vec != 0 || !aligned(w, 16)) return IQ_EINVAL;
+    if (batch > 1 && (w_batch_stride < (rows - 1) * ldw + cols || w_batch_stride % vec != 0)) return IQ_EINVAL;
     if (importance != nullptr) {
         if (!aligned(importance, 16) || imp_batch_stride < 0 || imp_batch_stride % 4 != 0) return IQ_EINVAL;
         if (batch > 1 && imp_batch_stride != 0 && imp_batch_stride < cols) return IQ_EINVAL;
@@ -94,6 +96,7 @@ iq_status iq_encode(const iq_desc* desc, const uint16_t* w, int64_t batch, int64
 
     iqk::EncodeParams p;
     p.w = w;
+    p.w_dtype = w_dtype;
     p.rows = rows;
     p.nblk = cols / 256;
     p.ldw = ldw;

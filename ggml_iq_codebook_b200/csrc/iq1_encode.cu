@@ -107,7 +107,7 @@ __device__ __forceinline__ void pack_block_m(uint8_t* out, int lane, int idx, in
     }
 }
 
-template <int FMT, int MODE, int K>
+template <int FMT, int MODE, int K, bool BF16IN>
 __global__ void __launch_bounds__(kWarps * 32, 2) iq1_encode_kernel(const EncodeParams p) {
     using Cfg = Iq1Cfg<FMT>;
     extern __shared__ __align__(16) char smem[];
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1_encode_kernel(const Encode
 
         // ---- load + validate (8 weights and importances per lane, 16-byte vector loads)
         float x[8], w[8];
-        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(p.w + e * p.w_bstride + r * p.ldw + blk * kBlock) + lane), x);
+        load_weights8<BF16IN>(p.w, p.w_dtype, e * p.w_bstride + r * p.ldw + blk * kBlock + 8 * lane, x);
         if (p.imp != nullptr) {
             const float4* ip = reinterpret_cast<const float4*>(p.imp + e * p.imp_bstride + blk * kBlock) + 2 * lane;
             const float4 a = __ldg(ip), c = __ldg(ip + 1);
@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1_encode_kernel(const Encode
 
 template <int FMT, int MODE, int K>
 cudaError_t launch_mode(const EncodeParams& p, int num_sms, cudaStream_t s) {
-    auto kern = iq1_encode_kernel<FMT, MODE, K>;
+    auto kern = p.w_dtype == IQ_IN_BF16 ? iq1_encode_kernel<FMT, MODE, K, true> : iq1_encode_kernel<FMT, MODE, K, false>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (err != cudaSuccess) return err;
     const int64_t ctas_needed = (p.nb + kWarps - 1) / kWarps;

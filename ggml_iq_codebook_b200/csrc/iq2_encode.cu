@@ -113,7 +113,7 @@ __device__ __forceinline__ void pack(uint8_t* out, int lane, int idx, uint32_t n
     else pack_block(out, lane, idx, neg, ls, d_half);
 }
 
-template <int FMT, int MODE, int K>
+template <int FMT, int MODE, int K, bool BF16IN>
 __global__ void __launch_bounds__(kWarps * 32, 2) iq2_encode_kernel(const EncodeParams p) {
     using Cfg = Iq2Cfg<FMT>;
     extern __shared__ __align__(16) char smem[];
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2_encode_kernel(const Encode
         const int64_t every_stride = p.nb * Cfg::BYTES;
 
         float x[8], w[8];
-        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(p.w + e * p.w_bstride + r * p.ldw + blk * kBlock) + lane), x);
+        load_weights8<BF16IN>(p.w, p.w_dtype, e * p.w_bstride + r * p.ldw + blk * kBlock + 8 * lane, x);
         if (p.imp != nullptr) {
             const float4* ip = reinterpret_cast<const float4*>(p.imp + e * p.imp_bstride + blk * kBlock) + 2 * lane;
             const float4 a = __ldg(ip), c = __ldg(ip + 1);
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2_encode_kernel(const Encode
 template <int FMT, int MODE, int K>
 cudaError_t launch_mode(const EncodeParams& p, int num_sms, cudaStream_t s) {
     constexpr int smem = Iq2Cfg<FMT>::SMEM;
-    auto kern = iq2_encode_kernel<FMT, MODE, K>;
+    auto kern = p.w_dtype == IQ_IN_BF16 ? iq2_encode_kernel<FMT, MODE, K, true> : iq2_encode_kernel<FMT, MODE, K, false>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     const int64_t ctas_needed = (p.nb + kWarps - 1) / kWarps;

@@ -9,7 +9,8 @@ namespace iqk {
 enum EncodeMode { kSearch = 0, kFixed = 1, kEvery = 2 };
 
 struct EncodeParams {
-    const uint16_t* w;
+    const void* w;
+    int w_dtype;  // IQ_IN_BF16, IQ_IN_F16 or IQ_IN_F32
     int64_t rows, nblk, ldw, w_bstride;
     const float* imp;  // nullptr: all ones
     int64_t imp_bstride;

@@ -60,6 +60,10 @@ typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3, IQ_FMT_IQ2
 
 typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 
+/* weight element types iq_encode takes (PR #2450: the encoders take fp32, f16 and bf16); each
+ * converts to fp32 exactly and the search runs on those values */
+typedef enum { IQ_IN_BF16 = 0, IQ_IN_F16 = 1, IQ_IN_F32 = 2 } iq_in_dtype;
+
 /* device-side findings, ORed into *flags */
 #define IQ_FLAG_NONFINITE 1u  /* a weight is NaN or +-inf                                 */
 #define IQ_FLAG_IMPORTANCE 2u /* an importance value is NaN, +-inf or negative            */
@@ -103,7 +107,8 @@ int32_t iq_choice_groups(int32_t fmt);
 int32_t iq_num_choices(int32_t fmt);
 
 /*
- * Encode `batch` weights of [rows, cols] bf16 (bit patterns as uint16).
+ * Encode `batch` weights of [rows, cols], elements of type w_dtype (IQ_IN_BF16 / IQ_IN_F16 bit
+ * patterns, or IQ_IN_F32 values).
  *   w[e * w_batch_stride + r * ldw + col]        (elements; ldw >= cols)
  *   importance: NULL (all ones) or fp32 per input column,
  *     importance[e * imp_batch_stride + col]     (imp_batch_stride 0 shares one vector)
@@ -141,12 +146,13 @@ int32_t iq_num_choices(int32_t fmt);
  * then the lower entry on equal error (PR #2595); a choice group's error is the sum of its two
  * groups'.
  * Without scales, amax == 0 or d rounding to fp16 zero gives the all-zero payload ([#2450]).
- * Alignment: w and importance 16-byte aligned, ldw and w_batch_stride multiples of 8 elements,
+ * Alignment: w and importance 16-byte aligned, ldw and w_batch_stride multiples of 16 bytes (8
+ * elements of bf16/f16, 4 of fp32),
  * imp_batch_stride a multiple of 4, payload and scales 2-byte aligned, grid 16-byte aligned
  * (IQ_EINVAL).
  */
-iq_status iq_encode(const iq_desc *desc, const uint16_t *w, int64_t batch, int64_t rows, int64_t cols,
-                    int64_t ldw, int64_t w_batch_stride, const float *importance,
+iq_status iq_encode(const iq_desc *desc, const void *w, int32_t w_dtype, int64_t batch, int64_t rows,
+                    int64_t cols, int64_t ldw, int64_t w_batch_stride, const float *importance,
                     int64_t imp_batch_stride, const uint8_t *choices, const uint16_t *scales,
                     int64_t scales_stride, int32_t every_choice, uint8_t *payload, uint32_t *flags, cudaStream_t stream);
 

@@ -177,7 +177,7 @@ def test_wrong_shapes_raise(dev, descs):
     with pytest.raises(iq.IQError):
         iq.iq_encode(descs["iq1_s"], torch.zeros((0, 256), dtype=torch.bfloat16, device=dev))
     with pytest.raises(iq.IQError):
-        iq.iq_encode(descs["iq1_s"], torch.zeros((4, 256), dtype=torch.float32, device=dev))
+        iq.iq_encode(descs["iq1_s"], torch.zeros((4, 256), dtype=torch.float64, device=dev))
 
 
 # --------------------------------------------------------------------------------- decode parity

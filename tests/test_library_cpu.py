@@ -59,30 +59,33 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     d = _desc()
     W = 0x10000  # a fake, 16-byte aligned address: validation must fail before it is touched
     # bad descriptors
-    assert E(None, W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(fmt=5)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(fmt=4, entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
+    assert E(None, W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=5)), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(fmt=4, entries=512)), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
              None) == 1
-    assert E(ctypes.byref(_desc(fmt=3, entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
+    assert E(ctypes.byref(_desc(fmt=3, entries=512)), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None,
              None) == 1
-    assert E(ctypes.byref(_desc(entries=512)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(anchor=float("nan"))), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(anchor=0.0)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(_desc(grid=0x1001)), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(entries=512)), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(anchor=float("nan"))), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(anchor=0.0)), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(_desc(grid=0x1001)), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
     # shapes: the [512, 384] case, empty tensors
-    assert E(ctypes.byref(d), W, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
-    assert E(ctypes.byref(d), W, 1, 0, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 2
-    assert E(ctypes.byref(d), W, 0, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 2
+    assert E(ctypes.byref(d), W, 0, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
+    assert E(ctypes.byref(d), W, 0, 1, 0, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 2
+    assert E(ctypes.byref(d), W, 0, 0, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 2
     # NULL buffers, strides, exclusive options
-    assert E(ctypes.byref(d), None, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(d), W, 1, 4, 256, 128, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(d), W + 2, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(d), W, 2, 4, 256, 256, 256, None, 0, None, None, 0, 0, W, None, None) == 1
-    assert E(ctypes.byref(d), W, 1, 4, 256, 256, 0, None, 0, W, None, 0, 1, W, None, None) == 1
-    assert E(ctypes.byref(d), W, 1, 4, 256, 256, 0, None, 0, None, None, 0, 2, W, None, None) == 1
+    assert E(ctypes.byref(d), None, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 0, 1, 4, 256, 128, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W + 2, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 0, 2, 4, 256, 256, 256, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 0, 1, 4, 256, 256, 0, None, 0, W, None, 0, 1, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 0, 1, 4, 256, 256, 0, None, 0, None, None, 0, 2, W, None, None) == 1
+    # weight dtypes: an unknown kind; f16 rows must be a multiple of 8 elements (fp32: 4)
+    assert E(ctypes.byref(d), W, 3, 1, 4, 256, 256, 0, None, 0, None, None, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 1, 1, 4, 256, 260, 0, None, 0, None, None, 0, 0, W, None, None) == 1
     # static scales: 2-byte aligned, stride >= 1
-    assert E(ctypes.byref(d), W, 1, 4, 256, 256, 0, None, 0, None, W + 1, 1, 0, W, None, None) == 1
-    assert E(ctypes.byref(d), W, 1, 4, 256, 256, 0, None, 0, None, W, 0, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 0, 1, 4, 256, 256, 0, None, 0, None, W + 1, 1, 0, W, None, None) == 1
+    assert E(ctypes.byref(d), W, 0, 1, 4, 256, 256, 0, None, 0, None, W, 0, 0, W, None, None) == 1
     # decode / choice search / sqrt_diag
     assert lib.iq_decode(ctypes.byref(d), W, 0, 1, W, None) == 2
     assert lib.iq_decode(ctypes.byref(d), W, 4, 7, W, None) == 1
@@ -92,7 +95,7 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert lib.iq_choice_search(ctypes.byref(d), W, 6, 1, 256, W, 4, W, 1, 0, W, W, 1, None, None) == 2  # 4 !| 6
     # IQ1_M: any anchor (it is derived per block); no choice search
     m = _desc(fmt=3, anchor=float("nan"))
-    assert E(ctypes.byref(m), W, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
+    assert E(ctypes.byref(m), W, 0, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
     assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None) == 4
     s2 = _desc(fmt=4, entries=1024, anchor=0.9)
     assert lib.iq_choice_search(ctypes.byref(s2), W, 0, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None) == 2
