@@ -1,7 +1,7 @@
 """CPU oracle for the GGML IQ encoder path -- TEST INFRASTRUCTURE ONLY.
 
 A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS / IQ2_S encoder and
-decoder, and the local-Hessian choice search (IQ1_S, IQ2_XS, IQ2_S), with this thin ctypes wrapper.
+decoder, and the local-Hessian choice search (all four formats), with this thin ctypes wrapper.
 It is the yardstick the CUDA library is checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import it; the library never does, and the two share no code.
 
@@ -189,7 +189,7 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
 
     w: [rows, cols], or [experts, rows, cols] with hess [experts, nblk, 256, 256] (each expert's
     rows use its own Hessian blocks); hess: [nblk, 256, 256] fp32 otherwise;
-    cand: [16, (experts,) rows, nblk, B] every-choice payloads.
+    cand: [C, (experts,) rows, nblk, B] every-choice payloads (C = 16; 8 for iq1_m).
     Returns (picks [(experts,) rows, nblk, G], payload [(experts,) rows, nblk, B]) and, with
     trace, the picks after step 2 and after each sweep [(experts,) rows, nblk, 3, G].
     Parity of the sweeps is pinned by the fp64 direct-objective replay in the tests.
@@ -203,7 +203,7 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     nblk = cols // 256
     G, B = CHOICE_GROUPS[fmt], BLOCK_BYTES[fmt]
     hess = np.ascontiguousarray(hess, dtype=np.float32).reshape(nexp, nblk, 256, 256)
-    cand = np.ascontiguousarray(cand, dtype=np.uint8).reshape(NUM_CHOICES, rows, nblk, B)
+    cand = np.ascontiguousarray(cand, dtype=np.uint8).reshape(CHOICES[fmt], rows, nblk, B)
     picks = np.zeros((rows, nblk, G), dtype=np.uint8)
     payload = np.zeros((rows, nblk, B), dtype=np.uint8)
     tr = np.zeros((rows, nblk, 3, G), dtype=np.uint8) if trace else None

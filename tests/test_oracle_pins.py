@@ -20,7 +20,7 @@ import pytest
 import torch
 
 import oracle
-from fp64_refs import (block_objective, iq1s_fields, iq1s_group_objectives, iq2s_fields, iq2xs_fields,
+from fp64_refs import (block_objective, iq1m_fields, iq1s_fields, iq1s_group_objectives, iq2s_fields, iq2xs_fields,
                        iq2xs_group_objectives, iq2xs_signs, replay_choice_search)
 from ggml_iq_codebook_b200 import synth
 
@@ -309,6 +309,8 @@ def _choices_of(fmt, p):
             out[i] = ls + 8 * neg
         elif fmt == "iq2_s":
             out[i] = iq2s_fields(p[i])[1]
+        elif fmt == "iq1_m":
+            out[i] = iq1m_fields(p[i])[1]
         else:
             out[i] = iq2xs_fields(p[i])[1]
     return out
@@ -368,7 +370,7 @@ def _deltas(fmt, grids, w, cand, r, b):
     return x[None] - xh
 
 
-@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m"])
 @pytest.mark.parametrize("offdiag", [0.02, 0.3])
 def test_choice_search_decisions_replay_in_fp64(grids, anchors, fmt, offdiag):
     """PR #3158: step 2 and both sweeps, checked decision by decision on the direct objective."""
@@ -389,7 +391,7 @@ def test_choice_search_decisions_replay_in_fp64(grids, anchors, fmt, offdiag):
         assert total_switches > 0  # the sweeps do something on correlated inputs
 
 
-@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m"])
 def test_choice_search_block_diagonal_hessian_makes_sweeps_noops(grids, anchors, fmt):
     G = oracle.CHOICE_GROUPS[fmt]
     W = 256 // G
@@ -401,7 +403,7 @@ def test_choice_search_block_diagonal_hessian_makes_sweeps_noops(grids, anchors,
     assert np.array_equal(trace[..., 0, :], trace[..., 2, :])
 
 
-@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m"])
 def test_choice_search_identity_hessian_keeps_encoder_choices(grids, anchors, fmt):
     """PR #3158: under H = I (with unit importance) the search keeps the encoder's own choices."""
     rows = 2 if fmt == "iq1_s" else 4
@@ -423,7 +425,7 @@ def test_choice_search_identity_hessian_keeps_encoder_choices(grids, anchors, fm
                 assert abs(a - bb) <= 1e-5 * max(a, bb), (r, g)  # only an fp near-tie may differ
 
 
-@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m"])
 def test_choice_search_payload_is_the_encode_under_picks(grids, anchors, fmt):
     """PR #3157 + #3158: the final payload equals quantize(..., choices=picks)."""
     w, hess, cand = _choice_case(fmt, grids, anchors, 3, 2, 131, 0.3)
