@@ -45,16 +45,17 @@ L2_FLUSH_BYTES = 256 << 20
 #     per 256-weight block: 32 groups x 2048 entries x 45 = 2,949,120 ops.
 #   IQ2_XS, per (group, entry): A and B chains (16) + 16 x (fma + min) = 48 ops;
 #     per block: 32 x 512 x 48 = 786,432 ops.
-#   Choice search (G choice groups of W = 256 / G columns, 16 choices), per row and block:
-#     own-block scores G x 16 x (W^2 + 2W - 1), gradient 256 x 256, two sweeps of
-#     G x 16 x (W^2 + 5W - 1) gains; gradient updates after a switch are data dependent and not
-#     counted. IQ2_XS and IQ2_S (G = 16): 310,528 ops; IQ1_S (G = 8): 507,520 ops.
+#   Choice search (G choice groups of W = 256 / G columns, C choices), per row and block:
+#     own-block scores G x C x (W^2 + 2W - 1), gradient 256 x 256, two sweeps of
+#     G x C x (W^2 + 5W - 1) gains; gradient updates after a switch are data dependent and not
+#     counted. IQ2_XS and IQ2_S (G = C = 16): 310,528 ops; IQ1_S (G = 8, C = 16): 507,520 ops;
+#     IQ1_M (G = 16, C = 8): 188,032 ops.
 #   IQ1_M runs IQ1_S's search (same 2048 x 16 candidates per group): 2,949,120 ops per block.
 #   IQ2_S runs IQ2_XS's per-entry work over 1024 entries: 32 x 1024 x 48 = 1,572,864 per block.
 OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120, "iq2_s": 1_572_864}
-def choice_ops_per_row_block(G: int) -> int:
+def choice_ops_per_row_block(G: int, C: int = 16) -> int:
     W = 256 // G
-    return G * 16 * (W * W + 2 * W - 1) + 256 * 256 + 2 * G * 16 * (W * W + 5 * W - 1)
+    return G * C * (W * W + 2 * W - 1) + 256 * 256 + 2 * G * C * (W * W + 5 * W - 1)
 SMS, FP32_LANES = 148, 128
 
 
@@ -200,6 +201,8 @@ class Workload:
             self._choice(synth.workload_choice_iq2xs(), "iq2_s")
         elif name == "choice_iq1s_4096x4096":
             self._choice(synth.workload_choice_iq2xs(), "iq1_s")
+        elif name == "choice_iq1m_4096x4096":
+            self._choice(synth.workload_choice_iq2xs(), "iq1_m")
         elif name == "choice_iq2xs_moe_16x1536x4096":
             self._choice(synth.workload_choice_moe(), "iq2_xs")
         elif name == "iq1s_decode_1m_blocks":
@@ -244,7 +247,7 @@ class Workload:
         nexp = lead[0] if len(lead) == 2 else 1
         self.imp = torch.empty((nexp, cols) if len(lead) == 2 else (cols,), dtype=torch.float32, device=self.dev)
         B, G = iq.BLOCK_BYTES[fmt], iq.CHOICE_GROUPS[fmt]
-        self.cand = torch.empty((16,) + lead + (nblk, B), dtype=torch.uint8, device=self.dev)
+        self.cand = torch.empty((iq.CHOICES[fmt],) + lead + (nblk, B), dtype=torch.uint8, device=self.dev)
         self.picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=self.dev)
         self.payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=self.dev)
         self.units = self.w.numel()
@@ -255,7 +258,7 @@ class Workload:
                      f"two-sweep search, {shape} bf16 N(0,0.02^2), one H = U^-1 U^-T per "
                      + ("expert and " if nexp > 1 else "") + "256-column block")
         self.dominant = "choice_search_kernel"
-        self.ops_per_launch = self.nblocks * choice_ops_per_row_block(G)
+        self.ops_per_launch = self.nblocks * choice_ops_per_row_block(G, iq.CHOICES[fmt])
         iq.iq_sqrt_diag(self.hess, out=self.imp)
         iq.iq_encode(self.desc[fmt], self.w, self.imp, every_choice=True, out=self.cand)
 
@@ -368,14 +371,16 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
     import oracle
     if name.startswith("choice_"):
         cfmt = {"choice_iq2xs_4096x4096": "iq2_xs", "choice_iq2s_4096x4096": "iq2_s",
-                "choice_iq1s_4096x4096": "iq1_s", "choice_iq2xs_moe_16x1536x4096": "iq2_xs"}[name]
+                "choice_iq1s_4096x4096": "iq1_s", "choice_iq1m_4096x4096": "iq1_m",
+                "choice_iq2xs_moe_16x1536x4096": "iq2_xs"}[name]
         if "moe" in name:  # the sample is the first rows of expert 0, under its own Hessians
             wl = synth.workload_choice_moe()
             w, hess = wl["w"][0], wl["hess"][0].numpy()
         else:
             wl = synth.workload_choice_iq2xs()
             w, hess = wl["w"], wl["hess"].numpy()
-        g = {"iq2_xs": synth.iq2xs_grid, "iq2_s": synth.iq2s_grid, "iq1_s": synth.iq1s_grid}[cfmt]()
+        g = {"iq2_xs": synth.iq2xs_grid, "iq2_s": synth.iq2s_grid, "iq1_s": synth.iq1s_grid,
+             "iq1_m": synth.iq1s_grid}[cfmt]()
         imp = oracle.sqrt_diag(hess)
 
         def run(r):

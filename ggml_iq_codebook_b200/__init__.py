@@ -223,7 +223,7 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     w: bf16 [rows, cols] with hess fp32 [cols/256, 256, 256], or a stack of experts
     [experts, rows, cols] with hess [experts, cols/256, 256, 256] (each expert's rows use its own
     Hessian blocks; the experts must be contiguous in the row dimension).
-    cand: uint8 [16, (experts,) rows, cols/256, B], the every-choice payloads.
+    cand: uint8 [C, (experts,) rows, cols/256, B], the every-choice payloads (C = CHOICES[fmt]).
     Returns (picks uint8 [(experts,) rows, cols/256, G], payload uint8 [(experts,) rows, cols/256, B]).
     """
     lib = load_library()
@@ -242,7 +242,7 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
     if not hess.is_contiguous() or hess.numel() != nexp * nblk * 256 * 256:
         raise IQError("hess must be contiguous [(experts,) cols/256, 256, 256]")
-    want = (NUM_CHOICES,) + lead + (nblk, B)
+    want = (CHOICES[fmt],) + lead + (nblk, B)
     if tuple(cand.shape) != want or not cand.is_contiguous():
         raise IQError(f"cand must be contiguous {want}")
     if picks is None:

@@ -141,7 +141,6 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
                            int64_t payload_ld, uint32_t* flags, cudaStream_t stream) {
     iq_status st = check_desc(desc);
     if (st != IQ_OK) return st;
-    if (desc->fmt == IQ_FMT_IQ1_M) return IQ_EUNSUPPORTED;
     if (w == nullptr || hess == nullptr || cand == nullptr || picks == nullptr || payload == nullptr)
         return IQ_EINVAL;
     if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;

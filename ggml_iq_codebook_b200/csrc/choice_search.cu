@@ -13,7 +13,8 @@
 // all 256 k; sums over i inside a group are a pairwise tree; gain = fma(2, t1, t2); switching
 // updates grad_i by an fma chain over the group's k. NaN and +inf scores never win.
 //
-// Formats: IQ1_S (8 groups of 32 columns), IQ2_XS and IQ2_S (16 groups of 16 columns); 16 choices.
+// Formats: IQ1_S (8 groups of 32 columns), IQ2_XS and IQ2_S (16 groups of 16 columns), 16 choices;
+// IQ1_M (16 groups of 16 columns, 8 choices: the other 8 lanes of a row never win).
 //
 // Experts: a stack of weights sharing a row layout runs in the same launch, row r taking Hessian
 // set r / rows_per_hess (PR #3218's reason for one launch: thousands of small expert weights).
@@ -48,16 +49,18 @@ __device__ __forceinline__ void load_vec(const float* src, float v[N]) {
     }
 }
 
-// The grid staged as 16-bit element codes: IQ1_S (+1 mask) | (-1 mask) << 8; IQ2_XS and IQ2_S
-// two bits (g - 1) / 2 per element.
+// The grid staged as 16-bit element codes: IQ1_S and IQ1_M (+1 mask) | (-1 mask) << 8; IQ2_XS and
+// IQ2_S two bits (g - 1) / 2 per element.
 template <int FMT>
 __device__ __forceinline__ uint16_t grid_code(int2 raw) {
     uint32_t c = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
-        if (FMT == IQ_FMT_IQ1_S) c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
-        else c |= (static_cast<uint32_t>((v - 1) >> 1) & 3u) << (2 * j);
+        if (FMT == IQ_FMT_IQ1_S || FMT == IQ_FMT_IQ1_M)
+            c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
+        else
+            c |= (static_cast<uint32_t>((v - 1) >> 1) & 3u) << (2 * j);
     }
     return static_cast<uint16_t>(c);
 }
@@ -68,6 +71,23 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
 // rounded exactly as the direct formula rounds it, and picked per element (no int-to-float).
 template <int FMT>
 __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid, int g, int grp8, float xh[8]) {
+    if (FMT == IQ_FMT_IQ1_M) {
+        // 56-byte layout: low index byte grp8; its nibble in byte 32 + grp8 / 2 (3 high index
+        // bits, bit 3 = delta -1/8); choice group g's 3-bit scale in word 48 + 2 (g / 4); d in
+        // the words' top nibbles
+        const uint16_t* pw = reinterpret_cast<const uint16_t*>(pc);
+        const float dm = half_bits_to_f32(iq1m_d_bits(pw[24], pw[25], pw[26], pw[27]));
+        const float s = __fmul_rn(dm, small_int_to_float(2u * ((static_cast<uint32_t>(pw[24 + (g >> 2)]) >> (3 * (g & 3))) & 7u) + 1u));
+        const uint32_t nib = (static_cast<uint32_t>(pc[32 + (grp8 >> 1)]) >> (4 * (grp8 & 1))) & 15u;
+        const float delta = (nib & 8u) ? -0.125f : 0.125f;
+        const float vp = __fmul_rn(s, __fadd_rn(1.0f, delta));
+        const float v0 = __fmul_rn(s, __fadd_rn(0.0f, delta));
+        const float vn = __fmul_rn(s, __fadd_rn(-1.0f, delta));
+        const uint32_t m = sgrid[static_cast<uint32_t>(pc[grp8]) | ((nib & 7u) << 8)];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xh[j] = ((m >> j) & 1u) ? vp : (((m >> (8 + j)) & 1u) ? vn : v0);
+        return;
+    }
     const float d = half_bits_to_f32(*reinterpret_cast<const uint16_t*>(pc));
     if (FMT == IQ_FMT_IQ2_S) {
         // 82-byte layout: low index byte 2 + grp8, sign byte 34 + grp8, 2 high index bits at
@@ -137,8 +157,12 @@ struct Cfg {
     static constexpr int RG = R / 4;                            // 4-row groups of the gradient tiles
     static constexpr int G = FMT == IQ_FMT_IQ1_S ? 8 : 16;     // choice groups per block
     static constexpr int W = kBlock / G;                        // columns per choice group
-    static constexpr int B = FMT == IQ_FMT_IQ1_S ? kIq1sBytes : FMT == IQ_FMT_IQ2_S ? kIq2sBytes : kIq2xsBytes;
-    static constexpr int E = FMT == IQ_FMT_IQ1_S ? kIq1sEntries : FMT == IQ_FMT_IQ2_S ? kIq2sEntries : kIq2xsEntries;
+    static constexpr int B = FMT == IQ_FMT_IQ1_S   ? kIq1sBytes
+                             : FMT == IQ_FMT_IQ1_M ? kIq1mBytes
+                             : FMT == IQ_FMT_IQ2_S ? kIq2sBytes
+                                                   : kIq2xsBytes;
+    static constexpr int E = FMT == IQ_FMT_IQ2_XS ? kIq2xsEntries : FMT == IQ_FMT_IQ2_S ? kIq2sEntries : kIq1sEntries;
+    static constexpr int NC = FMT == IQ_FMT_IQ1_M ? kIq1mChoices : kChoices;  // candidates per row
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
     // shared memory layout (bytes)
     static constexpr int oHp = 0;                                 // float [2][W][256], double buffer
@@ -246,7 +270,8 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     };
     prefetch(0);
 
-    // ---- stage the grid codes, the row's x (bf16) and its 16 candidate payloads
+    // ---- stage the grid codes, the row's x (bf16) and its candidate payloads (lanes past the
+    // format's NC candidates stage zeros and never win)
     for (int q = tid; q < C::E; q += kThreads) sgrid[q] = grid_code<FMT>(__ldg(reinterpret_cast<const int2*>(p.grid) + q));
     if (active) {
         const uint4* xs = reinterpret_cast<const uint4*>(p.w + row * p.ldw + blk * kBlock);
@@ -263,13 +288,18 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         if (__any_sync(hmask, nonfinite) && c == 0) raise_flags(p.flags, IQ_FLAG_NONFINITE);
         // 2-byte copies (B is even and the caller's candidates are 2-byte aligned), all loads
         // issued before the stores
-        const uint16_t* src = reinterpret_cast<const uint16_t*>(p.cand + c * p.cand_cstride + (row * p.cand_ld + blk) * C::B);
         uint16_t* dst = reinterpret_cast<uint16_t*>(cand + c * C::B);
-        uint16_t stage[C::B / 2];
+        if (c < C::NC) {
+            const uint16_t* src = reinterpret_cast<const uint16_t*>(p.cand + c * p.cand_cstride + (row * p.cand_ld + blk) * C::B);
+            uint16_t stage[C::B / 2];
 #pragma unroll
-        for (int i = 0; i < C::B / 2; ++i) stage[i] = __ldg(src + i);
+            for (int i = 0; i < C::B / 2; ++i) stage[i] = __ldg(src + i);
 #pragma unroll
-        for (int i = 0; i < C::B / 2; ++i) dst[i] = stage[i];
+            for (int i = 0; i < C::B / 2; ++i) dst[i] = stage[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < C::B / 2; ++i) dst[i] = 0;
+        }
     } else {
         for (int i = c; i < kBlock; i += 16) curT[i * kRows + hr] = 0.0f;
     }
@@ -309,7 +339,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
             group_matvec<W>(Hp, g * W, dl, v);
 #pragma unroll
             for (int i = 0; i < W; ++i) v[i] = __fmul_rn(dl[i], v[i]);
-            const float score = tree_sum<W>(v);
+            const float score = c < C::NC ? tree_sum<W>(v) : INFINITY;
             float best;
             int cstar;
             half_argmin(score, c, hmask, best, cstar);
@@ -378,7 +408,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
                     v[i] = __fmul_rn(u[i], v[i]);
                 }
                 const float t1 = tree_sum<W>(p1), t2 = tree_sum<W>(v);
-                gain = __fmaf_rn(2.0f, t1, t2);
+                gain = c < C::NC ? __fmaf_rn(2.0f, t1, t2) : INFINITY;
             }
             float best;
             int cstar;
@@ -454,7 +484,23 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         uint8_t* out = p.payload + (row * p.payload_ld + blk) * C::B;
         for (int i = c; i < C::B; i += 16) {
             uint8_t v;
-            if (i < 2) {
+            if (FMT == IQ_FMT_IQ1_M) {
+                if (i < 32) {  // low index byte of 8-weight group i: choice group i / 2
+                    v = cand[pick[i >> 1] * C::B + i];
+                } else if (i < 48) {  // the nibbles of choice group i - 32's two groups
+                    v = cand[pick[i - 32] * C::B + i];
+                } else {  // scale word q: choice groups 4q..4q+3 at shifts 0,3,6,9; d's nibble on top
+                    const int q = (i - 48) >> 1;
+                    uint32_t wv = (static_cast<uint32_t>(cand[49 + 2 * q]) << 8) & 0xF000u;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint8_t* pc = cand + pick[4 * q + j] * C::B;
+                        const uint32_t wj = static_cast<uint32_t>(pc[48 + 2 * q]) | (static_cast<uint32_t>(pc[49 + 2 * q]) << 8);
+                        wv |= wj & (7u << (3 * j));
+                    }
+                    v = static_cast<uint8_t>((i & 1) ? (wv >> 8) : wv);
+                }
+            } else if (i < 2) {
                 v = cand[i];
             } else if (FMT == IQ_FMT_IQ2_S) {
                 if (i < 66) {  // low index and sign bytes of 8-weight group q8: choice group q8 / 2
@@ -506,6 +552,7 @@ cudaError_t launch_choice_search(int fmt, const ChoiceParams& p, int /*num_sms*/
     if (p.rows == 0 || p.nblk == 0) return cudaSuccess;
     if (fmt == IQ_FMT_IQ1_S) return launch<IQ_FMT_IQ1_S>(p, s);
     if (fmt == IQ_FMT_IQ2_S) return launch<IQ_FMT_IQ2_S>(p, s);
+    if (fmt == IQ_FMT_IQ1_M) return launch<IQ_FMT_IQ1_M>(p, s);
     return launch<IQ_FMT_IQ2_XS>(p, s);
 }
 

@@ -167,8 +167,7 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
 
 /*
  * Local-Hessian choice search (PR #3158 steps; one fused launch as in PR #3218) for the first
- * nblk 256-column blocks of a [rows, ldw] bf16 weight. IQ1_S, IQ2_XS and IQ2_S (IQ1_M:
- * IQ_EUNSUPPORTED).
+ * nblk 256-column blocks of a [rows, ldw] bf16 weight, for every format (IQ1_M: 8 choices).
  *   hess: fp32 [rows / rows_per_hess][nblk][256][256], the symmetric diagonal blocks of the input
  *     Hessian, read as H[k][i] (row k, column i) for (H v)_i. Row r uses set r / rows_per_hess:
  *     a stack of experts that share a row layout runs in one call, each with its own Hessian
