@@ -13,8 +13,8 @@
 //           B = V_0 g_0,  then B = fma(V_j, g_j, B);   m = fma(s, A, B)
 //   argmin_g m (lowest entry on ties); e = s m_min; sub-block E = e_even + e_odd; argmin_ls E.
 //
-// IQ2_S (PR #2512 codec, PR #2565 CUDA encoder commit texts): a 1024-entry grid and a full 8-bit
-// sign mask per group, so the input's signs are kept (nothing is flipped) and a_j = |x_j|; the
+// IQ2_S (PR #2512 codec, PR #2565 CUDA encoder commit texts): a 1024-entry grid and eight sign
+// bits for each group, so the input's signs are kept (nothing is flipped) and a_j = |x_j|; the
 // 82-byte block holds d, the low index bytes, the sign bytes, the 2-bit high index fields (group
 // g at shift 2 (g % 4) of byte 66 + g/4) and the scale nibbles at bytes 74..81.
 //

@@ -8,14 +8,14 @@
  *     block is packed into its fixed byte layout. Sources: PR #2723 "Weight the IQ1 encoders by
  *     the square root of GPTQ's Hessian diagonal" (objective, delta = +-1/8, unweighted d);
  *     PR #2450 "[OMNIML-5899] Add IQ tests and release notes", review comments (IQ1_S 50-byte and
- *     IQ2_XS 74-byte layouts, d = fp16((amax / 16.875) * 0.61), 16-way choice, lowest index wins
- *     on equal error, even sign parity); the IQ2_S codec commit text on the PR #2525 page
- *     (IQ2_XS fixes parity by flipping the weakest element).
+ *     IQ2_XS 74-byte layouts, d = fp16((amax / 16.875) * 0.61), a choice among 16 with ties going
+ *     to the lower index, even sign parity); the IQ2_S codec commit text on the PR #2525 page
+ *     (IQ2_XS repairs an odd sign count at its weakest element).
  *   - fixed per-group choices (PR #3157) and the one-pass every-choice encode (PR #3159);
  *   - IQ1_M (PR #2513 codec and PR #2595 encoder commit texts): the IQ1_S search with a local
  *     scale per 16 weights, a delta per 8-weight group and d kept in four scale words;
  *   - IQ2_S (PR #2512 codec and PR #2565 encoder commit texts): the IQ2_XS search over a
- *     1024-entry grid with a full 8-bit sign mask per group (the input's signs, no parity flip);
+ *     1024-entry grid with eight sign bits for each group (the input's signs, no parity flip);
  *   - decoding of the four layouts;
  *   - the local-Hessian choice search (PR #3158, fused in PR #3218 "[4/4] Run the local-Hessian
  *     choice search as one CUDA kernel").

@@ -4,8 +4,8 @@ IQ1_M (PR #2513 codec and PR #2595 CUDA encoder commit texts, on the page of PR 
 shifted-grid search, a local scale per two groups, a delta per group, d stored as the top nibbles
 of four scale words, and the anchor clamp(0.58 + 0.035 * peak_to_rms, 0.65, 0.95). What fixes it:
 
-* the pages' own anchor test: blocks whose peak-to-RMS is exactly 1, 4, 8 and 16 reach both clamps
-  and two points on the slope, with d computed here in numpy's IEEE fp32/fp16;
+* the anchor points PR #2513's test uses: blocks built with peak-to-RMS ratios of 1, 4, 8 and 16
+  reach both clamps and two points on the slope, with d computed here in numpy's IEEE fp32/fp16;
 * a hand-built block decoded against values written out from the layout reading;
 * fp64 brute force: every pick reaches the minimum of the direct residual over (ls, delta, entry);
 * the tie order the pages state (lower shift, then lower entry), uniform-importance invariance,
@@ -37,7 +37,7 @@ def _enc(grids, w, **kw):
 
 @pytest.mark.parametrize("ratio,anchor_expected", [(1, 0.65), (4, 0.72), (8, 0.86), (16, 0.95)])
 def test_anchor_follows_peak_to_rms(grids, ratio, anchor_expected):
-    """PR #2513 pins the anchor at peak-to-RMS 1, 4, 8 and 16: both clamps and two slope points."""
+    """The anchor at peak-to-RMS 1, 4, 8 and 16 (PR #2513's test points): both clamps, two slope points."""
     n = 256 // (ratio * ratio)                       # n unit spikes in 256 weights: rms = sqrt(n/256)
     amax = 0.375
     x = np.zeros((1, 256), np.float32)

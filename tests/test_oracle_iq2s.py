@@ -1,8 +1,8 @@
 """Pins of the oracle's IQ2_S encoder and decoder (CPU only, no GPU).
 
 IQ2_S (PR #2512 codec and PR #2565 CUDA encoder commit texts, on the page of PR #2525): a
-1024-entry magnitude grid and a full 8-bit sign mask per group, so the encoder keeps the input's
-signs and searches magnitudes directly; a 4-bit local scale per 16 weights. What fixes it:
+1024-entry magnitude grid and eight sign bits for each group, so the encoder keeps the input's
+signs and searches the magnitudes alone; a 4-bit local scale per 16 weights. What fixes it:
 
 * a hand-built 82-byte block decoded against values written out from the layout reading;
 * every sign mask equals the input's sign bits (no parity flip, unlike IQ2_XS);

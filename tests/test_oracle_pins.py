@@ -270,7 +270,8 @@ def test_decode_is_exact(grids, anchors, fmt):
 
 @pytest.mark.parametrize("fmt", ["iq1_s", "iq2_xs"])
 def test_fixed_choices(grids, anchors, fmt):
-    """PR #3157: a fixed choice reproduces, group by group, the encode with that choice everywhere."""
+    """PR #3157: under fixed choices each group's fields equal those of the encode that forces its
+    choice on every group."""
     G = oracle.CHOICE_GROUPS[fmt]
     w, imp = _case(3, 512, 81)
     p, _ = oracle.encode(fmt, grids[fmt], anchors[fmt], w, importance=imp)
@@ -333,7 +334,7 @@ def test_zero_nonfinite_and_range_policy(grids, anchors, fmt):
     B = oracle.BLOCK_BYTES[fmt]
     w, imp = _case(6, 256, 91, weighted=True)
     w = w.clone()
-    w[1] = 0.0                        # all-zero block: canonical zero payload, no flag
+    w[1] = 0.0                        # all-zero block: all-zero payload, no flag
     w[2] = 1e-7                       # d underflows fp16: zero payload, no flag
     w[3, 17] = float("nan")           # non-finite weight
     w[4, 5] = float("inf")
@@ -487,7 +488,7 @@ def test_block_objective_is_quadratic_form():
 # ------------------------------------------------------------------------------ tie-breaks
 
 def test_iq1s_lowest_index_wins_on_equal_error(grids, anchors):
-    """PR #2450 review: 'lowest index wins on equal error'. With zero importance on two columns of
+    """PR #2450 review: on equal error the lower index is taken. With zero importance on two columns of
     each group, entries that differ only there tie exactly (also in fp64); the lowest must win.
     A sub-block with zero importance everywhere ties on every (entry, choice): choice 0, entry 0."""
     w, _ = _case(2, 256, 141, weighted=False)
