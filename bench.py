@@ -161,6 +161,35 @@ def weak_scaling_value(units_per_rank: int, world: int, ms_per_step_max: float) 
 
 # ------------------------------------------------------------------------------------ workloads
 
+# workload -> (format, weight shape, description): shared by both arms' JSON config
+def _choice_text(fmt: str, shape: str, experts: bool) -> str:
+    return (f"local-Hessian choice search, {fmt.upper()}: sqrt(diag H) + one-pass every-choice encode + "
+            f"two-sweep search, {shape} bf16 N(0,0.02^2), one H = U^-1 U^-T per "
+            + ("expert and " if experts else "") + "256-column block")
+
+
+WORKLOADS = {
+    "iq1s_4096x4096_weighted": ("iq1_s", [4096, 4096], "IQ1_S importance-weighted encode + bf16 decode, 4096x4096 "
+                                "bf16 N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))"),
+    "iq1m_4096x4096_weighted": ("iq1_m", [4096, 4096], "IQ1_M importance-weighted encode + bf16 decode, 4096x4096 "
+                                "bf16 N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))"),
+    "iq2s_8192x4096": ("iq2_s", [8192, 4096], "IQ2_S importance-weighted encode + bf16 decode, 8192x4096 bf16 "
+                       "N(0,0.015^2), importance lognormal(0,1)"),
+    "iq2xs_8192x4096": ("iq2_xs", [8192, 4096], "IQ2_XS importance-weighted encode + bf16 decode, 8192x4096 bf16 "
+                        "N(0,0.015^2), importance lognormal(0,1)"),
+    "iq1s_moe_256x1536x4096": ("iq1_s", [256, 1536, 4096], "IQ1_S weighted encode of 256 experts x 1536x4096 bf16 "
+                               "in one call + bf16 decode, importance lognormal(0,1) per expert"),
+    "iq1s_64x256": ("iq1_s", [64, 256], "IQ1_S encode + bf16 decode, one 64x256 bf16 weight, uniform importance"),
+    "choice_iq2xs_4096x4096": ("iq2_xs", [4096, 4096], _choice_text("iq2_xs", "4096x4096", False)),
+    "choice_iq2s_4096x4096": ("iq2_s", [4096, 4096], _choice_text("iq2_s", "4096x4096", False)),
+    "choice_iq1s_4096x4096": ("iq1_s", [4096, 4096], _choice_text("iq1_s", "4096x4096", False)),
+    "choice_iq1m_4096x4096": ("iq1_m", [4096, 4096], _choice_text("iq1_m", "4096x4096", False)),
+    "choice_iq2xs_moe_16x1536x4096": ("iq2_xs", [16, 1536, 4096], _choice_text("iq2_xs", "16x1536x4096", True)),
+    "iq1s_decode_1m_blocks": ("iq1_s", [4096, 4096], "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 "
+                              "weighted payload x16)"),
+}
+
+
 class Workload:
     """Inputs on the device plus one hot-path step; `units` weights per step."""
 
@@ -172,42 +201,26 @@ class Workload:
         self.desc = {"iq1_s": iq.make_desc("iq1_s", g1), "iq2_xs": iq.make_desc("iq2_xs", g2),
                      "iq1_m": iq.make_desc("iq1_m", g1), "iq2_s": iq.make_desc("iq2_s", g3)}
         self.launches_per_step = 2
+        if name not in WORKLOADS:
+            raise SystemExit(f"unknown workload {name}")
+        text = WORKLOADS[name][2]
         if name == "iq1s_4096x4096_weighted":
-            wl = synth.workload_iq1s_4096x4096_weighted()
-            self._encode_decode(wl, "IQ1_S importance-weighted encode + bf16 decode, 4096x4096 bf16 "
-                                    "N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))")
+            self._encode_decode(synth.workload_iq1s_4096x4096_weighted(), text)
         elif name == "iq1m_4096x4096_weighted":
-            wl = dict(synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m")
-            self._encode_decode(wl, "IQ1_M importance-weighted encode + bf16 decode, 4096x4096 bf16 "
-                                    "N(0,0.02^2) with 1% columns x8, importance sqrt(lognormal(0,1))")
+            self._encode_decode(dict(synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m"), text)
         elif name == "iq2s_8192x4096":
-            wl = dict(synth.workload_iq2xs_8192x4096(), fmt="iq2_s")
-            self._encode_decode(wl, "IQ2_S importance-weighted encode + bf16 decode, 8192x4096 bf16 "
-                                    "N(0,0.015^2), importance lognormal(0,1)")
+            self._encode_decode(dict(synth.workload_iq2xs_8192x4096(), fmt="iq2_s"), text)
         elif name == "iq2xs_8192x4096":
-            wl = synth.workload_iq2xs_8192x4096()
-            self._encode_decode(wl, "IQ2_XS importance-weighted encode + bf16 decode, 8192x4096 bf16 "
-                                    "N(0,0.015^2), importance lognormal(0,1)")
+            self._encode_decode(synth.workload_iq2xs_8192x4096(), text)
         elif name == "iq1s_moe_256x1536x4096":
-            wl = synth.workload_iq1s_moe(device=dev)
-            self._encode_decode(wl, "IQ1_S weighted encode of 256 experts x 1536x4096 bf16 in one call "
-                                    "+ bf16 decode, importance lognormal(0,1) per expert")
+            self._encode_decode(synth.workload_iq1s_moe(device=dev), text)
         elif name == "iq1s_64x256":
-            wl = synth.workload_iq1s_64x256()
-            self._encode_decode(wl, "IQ1_S encode + bf16 decode, one 64x256 bf16 weight, uniform importance")
-        elif name == "choice_iq2xs_4096x4096":
-            self._choice(synth.workload_choice_iq2xs(), "iq2_xs")
-        elif name == "choice_iq2s_4096x4096":
-            self._choice(synth.workload_choice_iq2xs(), "iq2_s")
-        elif name == "choice_iq1s_4096x4096":
-            self._choice(synth.workload_choice_iq2xs(), "iq1_s")
-        elif name == "choice_iq1m_4096x4096":
-            self._choice(synth.workload_choice_iq2xs(), "iq1_m")
-        elif name == "choice_iq2xs_moe_16x1536x4096":
-            self._choice(synth.workload_choice_moe(), "iq2_xs")
+            self._encode_decode(synth.workload_iq1s_64x256(), text)
+        elif name.startswith("choice_"):
+            wl = synth.workload_choice_moe() if "moe" in name else synth.workload_choice_iq2xs()
+            self._choice(wl, WORKLOADS[name][0], text)
         elif name == "iq1s_decode_1m_blocks":
-            wl = synth.workload_iq1s_4096x4096_weighted()
-            self._encode_decode(wl, "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 weighted payload x16)")
+            self._encode_decode(synth.workload_iq1s_4096x4096_weighted(), text)
             self.kind = "decode"
             self.payload = self.payload.reshape(-1, 50).repeat(16, 1)
             self.decoded = torch.empty((self.payload.shape[0], 256), dtype=torch.bfloat16, device=self.dev)
@@ -216,8 +229,6 @@ class Workload:
             self.launches_per_step = 1
             self.dominant = "decode_kernel"
             self.ops_per_launch = None
-        else:
-            raise SystemExit(f"unknown workload {name}")
 
     def _encode_decode(self, wl, text):
         self.fmt = wl["fmt"]
@@ -238,7 +249,7 @@ class Workload:
         # validate once (findings word + raise) before anything is timed
         iq.iq_encode(self.desc[self.fmt], self.w, self.imp, out=self.payload)
 
-    def _choice(self, wl, fmt):
+    def _choice(self, wl, fmt, text):
         self.fmt, self.kind = fmt, "choice"
         self.w_host, self.hess_host = wl["w"], wl["hess"]
         self.w, self.hess = wl["w"].to(self.dev), wl["hess"].to(self.dev)
@@ -253,10 +264,7 @@ class Workload:
         self.units = self.w.numel()
         self.nblocks = self.units // 256
         self.launches_per_step = 3
-        shape = "x".join(str(v) for v in self.w.shape)
-        self.text = (f"local-Hessian choice search, {fmt.upper()}: sqrt(diag H) + one-pass every-choice encode + "
-                     f"two-sweep search, {shape} bf16 N(0,0.02^2), one H = U^-1 U^-T per "
-                     + ("expert and " if nexp > 1 else "") + "256-column block")
+        self.text = text
         self.dominant = "choice_search_kernel"
         self.ops_per_launch = self.nblocks * choice_ops_per_row_block(G, iq.CHOICES[fmt])
         iq.iq_sqrt_diag(self.hess, out=self.imp)
@@ -424,8 +432,9 @@ def reference_arm(args, n_gpus, config):
     import oracle
     rate, rows, cols, dt, cores, run = oracle_sample_rate(args.workload, budget_s=1.0)
     # per step: a bounded sample sized so that warm-up + timed steps take about 90 s in all
+    budget = float(os.environ.get("IQ_BENCH_REFERENCE_SECONDS", "90"))
     per_row = dt / rows
-    rows = int(max(1, min(rows * 50, 90.0 / (args.steps + args.warmup) / per_row)))
+    rows = int(max(1, min(rows * 50, budget / (args.steps + args.warmup) / per_row)))
     for _ in range(args.warmup):
         run(rows)
     t0 = time.perf_counter()
@@ -461,8 +470,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     peaks = load_peaks()
+    if args.workload not in WORKLOADS:
+        raise SystemExit(f"unknown workload {args.workload}")
+    fmt, shape, text = WORKLOADS[args.workload]
     config = {"workload": args.workload, "l2": "flushed before every step (256 MiB write, outside the events)",
-              "parallelism": f"replicas x{world} (independent problems per rank)"}
+              "parallelism": f"replicas x{world} (independent problems per rank)", "format": fmt,
+              "shape": shape, "text": text}
 
     if args.impl == "reference":
         if rank == 0:
@@ -480,7 +493,6 @@ def main():
     torch.cuda.set_device(dev)
     iq.load_library()
     wl = Workload(args.workload, dev, peaks)
-    config.update({"format": wl.fmt, "shape": list(wl.w.shape), "text": wl.text})
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     for _ in range(args.warmup):

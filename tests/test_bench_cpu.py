@@ -37,3 +37,25 @@ def test_traffic_exact_scaled_and_stale(tmp_path, monkeypatch):
 def test_weak_scaling_value():
     assert bench.weak_scaling_value(16_777_216, 1, 7.0) == 16_777_216 / 7e-3 / 1e6
     assert bench.weak_scaling_value(100, 4, 2.0) == 4 * bench.weak_scaling_value(100, 1, 2.0)
+
+
+def test_workload_table():
+    import ggml_iq_codebook_b200 as iq
+    for name, (fmt, shape, text) in bench.WORKLOADS.items():
+        assert fmt in iq.IQ_FMT and shape[-1] % 256 == 0 and text, name
+
+
+def test_reference_arm_prints_the_contract_line():
+    """The oracle arm on the host cores (no GPU): one JSON line with the own arm's config."""
+    import json
+    import subprocess
+    env = dict(os.environ, IQ_BENCH_REFERENCE_SECONDS="2")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3",
+                          "--warmup", "3", "--workload", "iq1s_64x256"], capture_output=True, text=True,
+                         timeout=300, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads([ln for ln in out.stdout.splitlines() if ln.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 3
+    assert line["config"]["workload"] == "iq1s_64x256" and line["config"]["format"] == "iq1_s"
+    assert line["config"]["shape"] == [64, 256]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
