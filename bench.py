@@ -185,6 +185,8 @@ WORKLOADS = {
     "choice_iq1s_4096x4096": ("iq1_s", [4096, 4096], _choice_text("iq1_s", "4096x4096", False)),
     "choice_iq1m_4096x4096": ("iq1_m", [4096, 4096], _choice_text("iq1_m", "4096x4096", False)),
     "choice_iq2xs_moe_16x1536x4096": ("iq2_xs", [16, 1536, 4096], _choice_text("iq2_xs", "16x1536x4096", True)),
+    "choice_iq2xs_4096x4096_per_block": ("iq2_xs", [4096, 4096], _choice_text("iq2_xs", "4096x4096", False)
+                                         + ", the search as one call per 256-column block (16 calls)"),
     "iq1s_decode_1m_blocks": ("iq1_s", [4096, 4096], "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 "
                               "weighted payload x16)"),
 }
@@ -195,6 +197,7 @@ class Workload:
 
     def __init__(self, name: str, dev, peaks):
         self.name, self.dev, self.peaks = name, dev, peaks
+        self.per_block = False
         g1 = torch.from_numpy(synth.iq1s_grid()).to(dev)
         g2 = torch.from_numpy(synth.iq2xs_grid()).to(dev)
         g3 = torch.from_numpy(synth.iq2s_grid()).to(dev)
@@ -219,6 +222,9 @@ class Workload:
         elif name.startswith("choice_"):
             wl = synth.workload_choice_moe() if "moe" in name else synth.workload_choice_iq2xs()
             self._choice(wl, WORKLOADS[name][0], text)
+            if name.endswith("_per_block"):
+                self.per_block = True
+                self.launches_per_step = 2 + self.w.shape[-1] // 256
         elif name == "iq1s_decode_1m_blocks":
             self._encode_decode(synth.workload_iq1s_4096x4096_weighted(), text)
             self.kind = "decode"
@@ -260,6 +266,7 @@ class Workload:
         B, G = iq.BLOCK_BYTES[fmt], iq.CHOICE_GROUPS[fmt]
         self.cand = torch.empty((iq.CHOICES[fmt],) + lead + (nblk, B), dtype=torch.uint8, device=self.dev)
         self.picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=self.dev)
+        self.picks_b = torch.empty((nblk,) + lead + (1, G), dtype=torch.uint8, device=self.dev)
         self.payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=self.dev)
         self.units = self.w.numel()
         self.nblocks = self.units // 256
@@ -291,7 +298,13 @@ class Workload:
             iq.iq_encode(d, self.w, self.imp, every_choice=True, out=self.cand, flags=False)
             if ev is not None:
                 ev[0].record()
-            iq.iq_choice_search(d, self.w, self.hess, self.cand, picks=self.picks, payload=self.payload)
+            if self.per_block:  # one call per 256-column block, on views into the whole-weight tensors
+                for b in range(self.w.shape[-1] // 256):
+                    iq.iq_choice_search(d, self.w[:, 256 * b:256 * (b + 1)], self.hess[b:b + 1],
+                                        self.cand[:, :, b:b + 1], picks=self.picks_b[b],
+                                        payload=self.payload[:, b:b + 1])
+            else:
+                iq.iq_choice_search(d, self.w, self.hess, self.cand, picks=self.picks, payload=self.payload)
             if ev is not None:
                 ev[1].record()
 
@@ -314,7 +327,8 @@ class Workload:
             self.w.copy_(host["w"], non_blocking=True)
             self.hess.copy_(host["hess"], non_blocking=True)
             self.step()
-            host["picks"].copy_(self.picks, non_blocking=True)
+            picks = self.picks_b if self.per_block else self.picks
+            host["picks"].view(-1).copy_(picks.view(-1), non_blocking=True)
             host["payload"].copy_(self.payload, non_blocking=True)
 
     def host_buffers(self):
@@ -380,7 +394,7 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
     if name.startswith("choice_"):
         cfmt = {"choice_iq2xs_4096x4096": "iq2_xs", "choice_iq2s_4096x4096": "iq2_s",
                 "choice_iq1s_4096x4096": "iq1_s", "choice_iq1m_4096x4096": "iq1_m",
-                "choice_iq2xs_moe_16x1536x4096": "iq2_xs"}[name]
+                "choice_iq2xs_moe_16x1536x4096": "iq2_xs", "choice_iq2xs_4096x4096_per_block": "iq2_xs"}[name]
         if "moe" in name:  # the sample is the first rows of expert 0, under its own Hessians
             wl = synth.workload_choice_moe()
             w, hess = wl["w"][0], wl["hess"][0].numpy()

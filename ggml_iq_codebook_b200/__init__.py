@@ -215,6 +215,19 @@ def iq_decode(desc: IQDesc, payload: torch.Tensor, out_dtype: torch.dtype = torc
     return out
 
 
+def _blocks_ld(t: torch.Tensor, lead: tuple, nblk: int, B: int, name: str) -> int:
+    """Row stride in blocks of a [..., (experts,) rows, nblk, B] uint8 view whose blocks are
+    contiguous and whose rows (across experts too) are evenly spaced; raises otherwise."""
+    tail = lead + (nblk, B)
+    if t.dtype != torch.uint8 or tuple(t.shape[-len(tail):]) != tail:
+        raise IQError(f"{name} must be uint8 [..., {', '.join(map(str, tail))}]")
+    if t.stride(-1) != 1 or t.stride(-2) != B or t.stride(-3) % B != 0 or t.stride(-3) < nblk * B:
+        raise IQError(f"{name}: each block must be contiguous and each row's blocks adjacent")
+    if len(lead) == 2 and lead[0] > 1 and t.stride(-4) != lead[1] * t.stride(-3):
+        raise IQError(f"{name}: the experts' rows must be evenly spaced")
+    return t.stride(-3) // B
+
+
 def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor,
                      picks: torch.Tensor | None = None, payload: torch.Tensor | None = None,
                      flags: torch.Tensor | None = None, stream=None):
@@ -222,9 +235,12 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
 
     w: bf16 [rows, cols] with hess fp32 [cols/256, 256, 256], or a stack of experts
     [experts, rows, cols] with hess [experts, cols/256, 256, 256] (each expert's rows use its own
-    Hessian blocks; the experts must be contiguous in the row dimension).
+    Hessian blocks; the experts must be evenly spaced in the row dimension).
     cand: uint8 [C, (experts,) rows, cols/256, B], the every-choice payloads (C = CHOICES[fmt]).
-    Returns (picks uint8 [(experts,) rows, cols/256, G], payload uint8 [(experts,) rows, cols/256, B]).
+    w, cand and payload may be views (say one 256-column block of a wider weight and its slices):
+    rows need only be evenly spaced, each block contiguous.
+    Returns (picks uint8 [(experts,) rows, cols/256, G] contiguous, payload uint8
+    [(experts,) rows, cols/256, B]).
     """
     lib = load_library()
     fmt = _fmt_of(desc)
@@ -236,22 +252,25 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     lead, cols = tuple(w.shape[:-1]), w.shape[-1]
     nexp, rows_e = (lead[0], lead[1]) if w.dim() == 3 else (1, lead[0])
     if w.dim() == 3 and nexp > 1 and w.stride(0) != rows_e * w.stride(1):
-        raise IQError("the experts of w must be contiguous in the row dimension")
+        raise IQError("the experts of w must be evenly spaced in the row dimension")
     rows = nexp * rows_e
     nblk = cols // 256
     B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
     if not hess.is_contiguous() or hess.numel() != nexp * nblk * 256 * 256:
         raise IQError("hess must be contiguous [(experts,) cols/256, 256, 256]")
-    want = (CHOICES[fmt],) + lead + (nblk, B)
-    if tuple(cand.shape) != want or not cand.is_contiguous():
-        raise IQError(f"cand must be contiguous {want}")
+    if cand.dim() != len(lead) + 3 or cand.shape[0] != CHOICES[fmt]:
+        raise IQError(f"cand must be [{CHOICES[fmt]}, (experts,) rows, cols/256, {B}]")
+    cand_ld = _blocks_ld(cand, lead, nblk, B, "cand")
     if picks is None:
         picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=w.device)
+    elif picks.dtype != torch.uint8 or tuple(picks.shape) != lead + (nblk, G) or not picks.is_contiguous():
+        raise IQError(f"picks must be a contiguous uint8 tensor of shape {lead + (nblk, G)}")
     if payload is None:
         payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=w.device)
+    payload_ld = _blocks_ld(payload, lead, nblk, B, "payload")
     _check(lib.iq_choice_search(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(-2), hess.data_ptr(),
-                                rows_e, cand.data_ptr(), nblk, rows * nblk * B, picks.data_ptr(),
-                                payload.data_ptr(), nblk, None if flags is None else flags.data_ptr(),
+                                rows_e, cand.data_ptr(), cand_ld, cand.stride(0), picks.data_ptr(),
+                                payload.data_ptr(), payload_ld, None if flags is None else flags.data_ptr(),
                                 _stream(stream)))
     return picks, payload
 

@@ -290,6 +290,25 @@ def test_choice_search_over_a_stack_of_experts(dev, descs, grids, anchors, fmt):
         assert torch.equal(pe, picks[e]) and torch.equal(ye, pay[e])
 
 
+def test_choice_search_one_block_per_call(dev, descs, grids, anchors):
+    """The same search run as one call per 256-column block, on views into the whole-weight
+    tensors (the GPTQ-style calling pattern), gives the picks and payload of one call over all."""
+    fmt, rows, nblk = "iq2_xs", 37, 3
+    w, hess = _choice_case(fmt, rows, nblk, 541, 0.3)
+    wd, hd = w.to(dev), hess.to(dev)
+    cand = iq.iq_encode(descs[fmt], wd, iq.iq_sqrt_diag(hd), every_choice=True)
+    picks, pay = iq.iq_choice_search(descs[fmt], wd, hd, cand)
+    pay_b = torch.zeros_like(pay)
+    for b in range(nblk):
+        pk, _ = iq.iq_choice_search(descs[fmt], wd[:, 256 * b:256 * (b + 1)], hd[b:b + 1], cand[:, :, b:b + 1],
+                                    payload=pay_b[:, b:b + 1])
+        assert torch.equal(pk[:, 0], picks[:, b])
+    assert torch.equal(pay_b, pay)
+    with pytest.raises(iq.IQError):                   # a payload buffer of the wrong shape is refused
+        iq.iq_choice_search(descs[fmt], wd, hd, cand, payload=torch.empty((rows, nblk, 73), dtype=torch.uint8,
+                                                                          device=dev))
+
+
 # --------------------------------------------------------------------------------- full sizes
 
 def _sample_rows(rows, k, seed):
