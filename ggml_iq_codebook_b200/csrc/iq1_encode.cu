@@ -226,136 +226,135 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1_encode_kernel(const Encode
 #pragma unroll
         for (int ls = 0; ls < 8; ++ls) s[ls] = __fmul_rn(d, static_cast<float>(2 * ls + 1));
 
-        if (MODE == kFixed && Cfg::M) {
-            // The lane's local scale is given; both deltas are searched, each keeping its lowest
-            // entry, and the negative shift wins only with a strictly smaller m.
-            float sv = s[0];
+        if constexpr (MODE == kFixed) {
+            if constexpr (Cfg::M) {
+                // The lane's local scale is given; both deltas are searched, each keeping its lowest
+                // entry, and the negative shift wins only with a strictly smaller m.
+                float sv = s[0];
 #pragma unroll
-            for (int ls = 1; ls < 8; ++ls) if (fixed_c == ls) sv = s[ls];
-            float bp = INFINITY, bn = INFINITY;
-            int qp = 0, qn = 0;
+                for (int ls = 1; ls < 8; ++ls) if (fixed_c == ls) sv = s[ls];
+                float bp = INFINITY, bn = INFINITY;
+                int qp = 0, qn = 0;
 #pragma unroll 4
-            for (int q = 0; q < kIq1sEntries; ++q) {
-                const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
-                const float mp = __fmaf_rn(sv, tm.Ap, tm.Cp), mn = __fmaf_rn(sv, tm.An, tm.Cn);
-                if (mp < bp) { bp = mp; qp = q; }
-                if (mn < bn) { bn = mn; qn = q; }
-            }
-            const int neg = bn < bp;
-            pack_block_m(out, lane, neg ? qn : qp, fixed_c, neg, d_half);
-            continue;
-        }
-        if (MODE == kFixed) {
-            // One choice per lane: direct argmin with the index (lowest entry on ties).
-            float sv = s[0];
-#pragma unroll
-            for (int ls = 1; ls < 8; ++ls) if ((fixed_c & 7) == ls) sv = s[ls];
-            const bool negd = fixed_c >= 8;
-            float best = INFINITY;
-            int bi = 0;
-#pragma unroll 4
-            for (int q = 0; q < kIq1sEntries; ++q) {
-                const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
-                const float m = negd ? __fmaf_rn(sv, tm.An, tm.Cn) : __fmaf_rn(sv, tm.Ap, tm.Cp);
-                if (m < best) { best = m; bi = q; }
-            }
-            pack_block(out, lane, bi, fixed_c, d_half);
-            continue;
-        }
-
-        // ---- search: running minima per choice, chunk of first appearance
-        float best[kChoices];
-        int bch[kChoices];
-#pragma unroll
-        for (int c = 0; c < kChoices; ++c) { best[c] = INFINITY; bch[c] = 0; }
-        for (int ch = 0; ch < kIq1sEntries / K; ++ch) {
-            float cm[kChoices];
-            {
-                const Terms ta = entry_terms(smem, lane_base, sgrid[ch * K], W, Tall);
-                const Terms tb = entry_terms(smem, lane_base, sgrid[ch * K + 1], W, Tall);
-#pragma unroll
-                for (int ls = 0; ls < 8; ++ls) {
-                    cm[ls] = fminf(__fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
-                    cm[8 + ls] = fminf(__fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
+                for (int q = 0; q < kIq1sEntries; ++q) {
+                    const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+                    const float mp = __fmaf_rn(sv, tm.Ap, tm.Cp), mn = __fmaf_rn(sv, tm.An, tm.Cn);
+                    if (mp < bp) { bp = mp; qp = q; }
+                    if (mn < bn) { bn = mn; qn = q; }
                 }
+                const int neg = bn < bp;
+                pack_block_m(out, lane, neg ? qn : qp, fixed_c, neg, d_half);
+            } else {
+                // One choice per lane: direct argmin with the index (lowest entry on ties).
+                float sv = s[0];
+#pragma unroll
+                for (int ls = 1; ls < 8; ++ls) if ((fixed_c & 7) == ls) sv = s[ls];
+                const bool negd = fixed_c >= 8;
+                float best = INFINITY;
+                int bi = 0;
+#pragma unroll 4
+                for (int q = 0; q < kIq1sEntries; ++q) {
+                    const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+                    const float m = negd ? __fmaf_rn(sv, tm.An, tm.Cn) : __fmaf_rn(sv, tm.Ap, tm.Cp);
+                    if (m < best) { best = m; bi = q; }
+                }
+                pack_block(out, lane, bi, fixed_c, d_half);
             }
+        } else {
+            // ---- search: running minima per choice, chunk of first appearance
+            float best[kChoices];
+            int bch[kChoices];
+#pragma unroll
+            for (int c = 0; c < kChoices; ++c) { best[c] = INFINITY; bch[c] = 0; }
+            for (int ch = 0; ch < kIq1sEntries / K; ++ch) {
+                float cm[kChoices];
+                {
+                    const Terms ta = entry_terms(smem, lane_base, sgrid[ch * K], W, Tall);
+                    const Terms tb = entry_terms(smem, lane_base, sgrid[ch * K + 1], W, Tall);
+#pragma unroll
+                    for (int ls = 0; ls < 8; ++ls) {
+                        cm[ls] = fminf(__fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
+                        cm[8 + ls] = fminf(__fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
+                    }
+                }
 #pragma unroll 2
-            for (int q = ch * K + 2; q < ch * K + K; q += 2) {
-                const Terms ta = entry_terms(smem, lane_base, sgrid[q], W, Tall);
-                const Terms tb = entry_terms(smem, lane_base, sgrid[q + 1], W, Tall);
+                for (int q = ch * K + 2; q < ch * K + K; q += 2) {
+                    const Terms ta = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+                    const Terms tb = entry_terms(smem, lane_base, sgrid[q + 1], W, Tall);
 #pragma unroll
-                for (int ls = 0; ls < 8; ++ls) {
-                    cm[ls] = min3f(cm[ls], __fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
-                    cm[8 + ls] = min3f(cm[8 + ls], __fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
+                    for (int ls = 0; ls < 8; ++ls) {
+                        cm[ls] = min3f(cm[ls], __fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
+                        cm[8 + ls] = min3f(cm[8 + ls], __fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < kChoices; ++c) {
+                    if (cm[c] < best[c]) { best[c] = cm[c]; bch[c] = ch; }
                 }
             }
-#pragma unroll
-            for (int c = 0; c < kChoices; ++c) {
-                if (cm[c] < best[c]) { best[c] = cm[c]; bch[c] = ch; }
-            }
-        }
 
-        // Recover the first entry of choice c that reached best[c] (0 if nothing beat +inf).
-        auto entry_of = [&](int c) -> int {
-            float target = best[0];
-            int ch = bch[0];
-            float sv = s[0];
+            // Recover the first entry of choice c that reached best[c] (0 if nothing beat +inf).
+            auto entry_of = [&](int c) -> int {
+                float target = best[0];
+                int ch = bch[0];
+                float sv = s[0];
 #pragma unroll
-            for (int k = 1; k < kChoices; ++k) if (k == c) { target = best[k]; ch = bch[k]; }
+                for (int k = 1; k < kChoices; ++k) if (k == c) { target = best[k]; ch = bch[k]; }
 #pragma unroll
-            for (int ls = 1; ls < 8; ++ls) if ((c & 7) == ls) sv = s[ls];
-            if (!(target < INFINITY)) return 0;
-            const bool negd = c >= 8;
-            for (int q = ch * K; q < ch * K + K; ++q) {
-                const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
-                const float m = negd ? __fmaf_rn(sv, tm.An, tm.Cn) : __fmaf_rn(sv, tm.Ap, tm.Cp);
-                if (m == target) return q;
-            }
-            return ch * K;  // not reached: the same arithmetic reproduces target
-        };
+                for (int ls = 1; ls < 8; ++ls) if ((c & 7) == ls) sv = s[ls];
+                if (!(target < INFINITY)) return 0;
+                const bool negd = c >= 8;
+                for (int q = ch * K; q < ch * K + K; ++q) {
+                    const Terms tm = entry_terms(smem, lane_base, sgrid[q], W, Tall);
+                    const float m = negd ? __fmaf_rn(sv, tm.An, tm.Cn) : __fmaf_rn(sv, tm.Ap, tm.Cp);
+                    if (m == target) return q;
+                }
+                return ch * K;  // not reached: the same arithmetic reproduces target
+            };
 
-        if (Cfg::M) {
-            // per ls: the group's delta (bit ls of negmask: -1/8 only with a strictly smaller m)
-            uint32_t negmask = 0;
+            if (Cfg::M) {
+                // per ls: the group's delta (bit ls of negmask: -1/8 only with a strictly smaller m)
+                uint32_t negmask = 0;
 #pragma unroll
-            for (int ls = 0; ls < kIq1mChoices; ++ls) negmask |= static_cast<uint32_t>(best[8 + ls] < best[ls]) << ls;
-            if (MODE == kEvery) {
+                for (int ls = 0; ls < kIq1mChoices; ++ls) negmask |= static_cast<uint32_t>(best[8 + ls] < best[ls]) << ls;
+                if (MODE == kEvery) {
+                    for (int ls = 0; ls < kIq1mChoices; ++ls) {
+                        const int neg = (negmask >> ls) & 1;
+                        pack_block_m(out + ls * every_stride, lane, entry_of(ls + 8 * neg), ls, neg, d_half);
+                    }
+                    continue;
+                }
+                // e = s m under the group's delta, E = e_even + e_odd over the choice group
+                int lstar = 0;
+                float bestE = INFINITY;
+#pragma unroll
                 for (int ls = 0; ls < kIq1mChoices; ++ls) {
-                    const int neg = (negmask >> ls) & 1;
-                    pack_block_m(out + ls * every_stride, lane, entry_of(ls + 8 * neg), ls, neg, d_half);
+                    const float mm = ((negmask >> ls) & 1) ? best[8 + ls] : best[ls];
+                    const float e = __fmul_rn(s[ls], mm);
+                    const float E = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 1));
+                    if (E < bestE) { bestE = E; lstar = ls; }
                 }
+                const int neg = (negmask >> lstar) & 1;
+                pack_block_m(out, lane, entry_of(lstar + 8 * neg), lstar, neg, d_half);
                 continue;
             }
-            // e = s m under the group's delta, E = e_even + e_odd over the choice group
-            int lstar = 0;
+            if (MODE == kEvery) {
+                for (int c = 0; c < kChoices; ++c) pack_block(out + c * every_stride, lane, entry_of(c), c, d_half);
+                continue;
+            }
+
+            // group errors, sub-block sums over the 4 lanes of a sub-block, choice argmin
+            int cstar = 0;
             float bestE = INFINITY;
 #pragma unroll
-            for (int ls = 0; ls < kIq1mChoices; ++ls) {
-                const float mm = ((negmask >> ls) & 1) ? best[8 + ls] : best[ls];
-                const float e = __fmul_rn(s[ls], mm);
-                const float E = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 1));
-                if (E < bestE) { bestE = E; lstar = ls; }
+            for (int c = 0; c < kChoices; ++c) {
+                const float e0 = __fmul_rn(s[c & 7], best[c]);
+                const float t2 = __fadd_rn(e0, __shfl_xor_sync(0xffffffffu, e0, 1));
+                const float E = __fadd_rn(t2, __shfl_xor_sync(0xffffffffu, t2, 2));
+                if (E < bestE) { bestE = E; cstar = c; }
             }
-            const int neg = (negmask >> lstar) & 1;
-            pack_block_m(out, lane, entry_of(lstar + 8 * neg), lstar, neg, d_half);
-            continue;
-        }
-        if (MODE == kEvery) {
-            for (int c = 0; c < kChoices; ++c) pack_block(out + c * every_stride, lane, entry_of(c), c, d_half);
-            continue;
-        }
-
-        // group errors, sub-block sums over the 4 lanes of a sub-block, choice argmin
-        int cstar = 0;
-        float bestE = INFINITY;
-#pragma unroll
-        for (int c = 0; c < kChoices; ++c) {
-            const float e0 = __fmul_rn(s[c & 7], best[c]);
-            const float t2 = __fadd_rn(e0, __shfl_xor_sync(0xffffffffu, e0, 1));
-            const float E = __fadd_rn(t2, __shfl_xor_sync(0xffffffffu, t2, 2));
-            if (E < bestE) { bestE = E; cstar = c; }
-        }
         pack_block(out, lane, entry_of(cstar), cstar, d_half);
+        }
     }
 }
 

@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2_encode_kernel(const Encode
 #pragma unroll
         for (int ls = 0; ls < 16; ++ls) s[ls] = __fmul_rn(d, static_cast<float>(2 * ls + 1));
 
-        if (MODE == kFixed) {
+        if constexpr (MODE == kFixed) {
             float sv = s[0];
 #pragma unroll
             for (int ls = 1; ls < 16; ++ls) if (fixed_c == ls) sv = s[ls];
@@ -232,73 +232,72 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq2_encode_kernel(const Encode
                 if (m < best) { best = m; bi = q; }
             }
             pack<FMT>(out, lane, bi, neg, fixed_c, d_half);
-            continue;
-        }
-
-        float best[kChoices];
-        int bch[kChoices];
+        } else {
+            float best[kChoices];
+            int bch[kChoices];
 #pragma unroll
-        for (int c = 0; c < kChoices; ++c) { best[c] = INFINITY; bch[c] = 0; }
-        for (int ch = 0; ch < Cfg::E / K; ++ch) {
-            float cm[kChoices];
-            {
-                Entry ea, eb;
-                load_entry(sg, ch * K, ea);
-                load_entry(sg, ch * K + 1, eb);
-                float Aa, Ba, Ab, Bb;
-                entry_AB(ea, w, V, Aa, Ba);
-                entry_AB(eb, w, V, Ab, Bb);
+            for (int c = 0; c < kChoices; ++c) { best[c] = INFINITY; bch[c] = 0; }
+            for (int ch = 0; ch < Cfg::E / K; ++ch) {
+                float cm[kChoices];
+                {
+                    Entry ea, eb;
+                    load_entry(sg, ch * K, ea);
+                    load_entry(sg, ch * K + 1, eb);
+                    float Aa, Ba, Ab, Bb;
+                    entry_AB(ea, w, V, Aa, Ba);
+                    entry_AB(eb, w, V, Ab, Bb);
 #pragma unroll
-                for (int c = 0; c < kChoices; ++c) cm[c] = fminf(__fmaf_rn(s[c], Aa, Ba), __fmaf_rn(s[c], Ab, Bb));
-            }
+                    for (int c = 0; c < kChoices; ++c) cm[c] = fminf(__fmaf_rn(s[c], Aa, Ba), __fmaf_rn(s[c], Ab, Bb));
+                }
 #pragma unroll 1
-            for (int q = ch * K + 2; q < ch * K + K; q += 2) {
-                Entry ea, eb;
-                load_entry(sg, q, ea);
-                load_entry(sg, q + 1, eb);
-                float Aa, Ba, Ab, Bb;
-                entry_AB(ea, w, V, Aa, Ba);
-                entry_AB(eb, w, V, Ab, Bb);
+                for (int q = ch * K + 2; q < ch * K + K; q += 2) {
+                    Entry ea, eb;
+                    load_entry(sg, q, ea);
+                    load_entry(sg, q + 1, eb);
+                    float Aa, Ba, Ab, Bb;
+                    entry_AB(ea, w, V, Aa, Ba);
+                    entry_AB(eb, w, V, Ab, Bb);
 #pragma unroll
-                for (int c = 0; c < kChoices; ++c)
-                    cm[c] = min3f(cm[c], __fmaf_rn(s[c], Aa, Ba), __fmaf_rn(s[c], Ab, Bb));
+                    for (int c = 0; c < kChoices; ++c)
+                        cm[c] = min3f(cm[c], __fmaf_rn(s[c], Aa, Ba), __fmaf_rn(s[c], Ab, Bb));
+                }
+#pragma unroll
+                for (int c = 0; c < kChoices; ++c) {
+                    if (cm[c] < best[c]) { best[c] = cm[c]; bch[c] = ch; }
+                }
             }
+
+            auto entry_of = [&](int c) -> int {
+                float target = best[0], sv = s[0];
+                int ch = bch[0];
+#pragma unroll
+                for (int k = 1; k < kChoices; ++k) if (k == c) { target = best[k]; ch = bch[k]; sv = s[k]; }
+                if (!(target < INFINITY)) return 0;
+                for (int q = ch * K; q < ch * K + K; ++q) {
+                    Entry en;
+                    load_entry_packed(sgp, q, en);
+                    float A, B;
+                    entry_AB(en, w, V, A, B);
+                    if (__fmaf_rn(sv, A, B) == target) return q;
+                }
+                return ch * K;  // not reached: the same arithmetic reproduces target
+            };
+
+            if (MODE == kEvery) {
+                for (int c = 0; c < kChoices; ++c) pack<FMT>(out + c * every_stride, lane, entry_of(c), neg, c, d_half);
+                continue;
+            }
+
+            int cstar = 0;
+            float bestE = INFINITY;
 #pragma unroll
             for (int c = 0; c < kChoices; ++c) {
-                if (cm[c] < best[c]) { best[c] = cm[c]; bch[c] = ch; }
+                const float e0 = __fmul_rn(s[c], best[c]);
+                const float E = __fadd_rn(e0, __shfl_xor_sync(0xffffffffu, e0, 1));
+                if (E < bestE) { bestE = E; cstar = c; }
             }
+            pack<FMT>(out, lane, entry_of(cstar), neg, cstar, d_half);
         }
-
-        auto entry_of = [&](int c) -> int {
-            float target = best[0], sv = s[0];
-            int ch = bch[0];
-#pragma unroll
-            for (int k = 1; k < kChoices; ++k) if (k == c) { target = best[k]; ch = bch[k]; sv = s[k]; }
-            if (!(target < INFINITY)) return 0;
-            for (int q = ch * K; q < ch * K + K; ++q) {
-                Entry en;
-                load_entry_packed(sgp, q, en);
-                float A, B;
-                entry_AB(en, w, V, A, B);
-                if (__fmaf_rn(sv, A, B) == target) return q;
-            }
-            return ch * K;  // not reached: the same arithmetic reproduces target
-        };
-
-        if (MODE == kEvery) {
-            for (int c = 0; c < kChoices; ++c) pack<FMT>(out + c * every_stride, lane, entry_of(c), neg, c, d_half);
-            continue;
-        }
-
-        int cstar = 0;
-        float bestE = INFINITY;
-#pragma unroll
-        for (int c = 0; c < kChoices; ++c) {
-            const float e0 = __fmul_rn(s[c], best[c]);
-            const float E = __fadd_rn(e0, __shfl_xor_sync(0xffffffffu, e0, 1));
-            if (E < bestE) { bestE = E; cstar = c; }
-        }
-        pack<FMT>(out, lane, entry_of(cstar), neg, cstar, d_half);
     }
 }
 
