@@ -58,7 +58,7 @@ def _load(path: str | None = None):
         lib.orc_decode.restype = None
         lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
         lib.orc_choice_search.restype = None
-        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, i64, P, P, P, P]
+        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, i64, P, P, P, P, P]
         lib.orc_sqrt_diag.restype = None
         lib.orc_sqrt_diag.argtypes = [P, i64, P]
         lib.orc_f32_to_f16.restype = ctypes.c_uint16
@@ -184,14 +184,16 @@ def decode(fmt: str, grid: np.ndarray, payload: np.ndarray) -> np.ndarray:
     return out
 
 
-def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False):
+def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False,
+                  objective=False):
     """Local-Hessian choice search over every 256-column block of w.
 
     w: [rows, cols], or [experts, rows, cols] with hess [experts, nblk, 256, 256] (each expert's
     rows use its own Hessian blocks); hess: [nblk, 256, 256] fp32 otherwise;
     cand: [C, (experts,) rows, nblk, B] every-choice payloads (C = 16; 8 for iq1_m).
     Returns (picks [(experts,) rows, nblk, G], payload [(experts,) rows, nblk, B]) and, with
-    trace, the picks after step 2 and after each sweep [(experts,) rows, nblk, 3, G].
+    trace, the picks after step 2 and after each sweep [(experts,) rows, nblk, 3, G]; with objective
+    (last), each row-block's final Delta^T H Delta [(experts,) rows, nblk] fp32.
     Parity of the sweeps is pinned by the fp64 direct-objective replay in the tests.
     """
     wb = _bf16_bits(w)
@@ -207,13 +209,16 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     picks = np.zeros((rows, nblk, G), dtype=np.uint8)
     payload = np.zeros((rows, nblk, B), dtype=np.uint8)
     tr = np.zeros((rows, nblk, 3, G), dtype=np.uint8) if trace else None
+    obj = np.zeros((rows, nblk), dtype=np.float32) if objective else None
     _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
                               rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
-                              _ptr(payload), _ptr(tr))
-    picks, payload = picks.reshape(lead + (nblk, G)), payload.reshape(lead + (nblk, B))
+                              _ptr(payload), _ptr(tr), _ptr(obj))
+    out = [picks.reshape(lead + (nblk, G)), payload.reshape(lead + (nblk, B))]
     if trace:
-        return picks, payload, tr.reshape(lead + (nblk, 3, G))
-    return picks, payload
+        out.append(tr.reshape(lead + (nblk, 3, G)))
+    if objective:
+        out.append(obj.reshape(lead + (nblk,)))
+    return tuple(out)
 
 
 def sqrt_diag(hess: np.ndarray) -> np.ndarray:

@@ -464,6 +464,22 @@ def test_choice_search_experts_use_their_own_hessians(grids, anchors, fmt):
     assert not np.array_equal(other, picks)           # the Hessians do reach the decisions
 
 
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m"])
+def test_choice_search_objective_is_the_final_quadratic_form(grids, anchors, fmt):
+    """The reported objective, sum_i Delta_i grad_i with the incrementally updated gradient,
+    equals Delta^T H Delta of the final payload recomputed in fp64 from scratch."""
+    w, hess, cand = _choice_case(fmt, grids, anchors, 4, 2, 151, 0.3)
+    picks, payload, obj = oracle.choice_search(fmt, grids[fmt], w, hess, cand, objective=True)
+    xh = oracle.decode(fmt, grids[fmt], payload).astype(np.float64)           # [rows, nblk, 256]
+    x = w.double().numpy().reshape(4, 2, 256)
+    for r in range(4):
+        for b in range(2):
+            dl = x[r, b] - xh[r, b]
+            H = hess[b].astype(np.float64)
+            scale = np.abs(dl) @ np.abs(H) @ np.abs(dl)
+            assert abs(float(obj[r, b]) - dl @ H @ dl) <= 1e-5 * scale, (r, b)
+
+
 def test_sqrt_diag_matches_numpy():
     h = torch.stack([synth.block_hessian(7), synth.block_hessian(8)]).numpy()
     want = np.sqrt(np.stack([np.diag(h[0]), np.diag(h[1])]).astype(np.float32)).reshape(-1)
