@@ -69,7 +69,8 @@ def load_library(path: str = LIB_PATH):
     lib.iq_decode.restype = ctypes.c_int
     lib.iq_decode.argtypes = [ctypes.POINTER(IQDesc), P, i64, i32, P, P]
     lib.iq_choice_search.restype = ctypes.c_int
-    lib.iq_choice_search.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, i64, P, i64, i64, P, P, i64, P, P]
+    lib.iq_choice_search.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, i64, P, i64, i64, P, P, i64, P, P,
+                                     P]
     lib.iq_sqrt_diag.restype = ctypes.c_int
     lib.iq_sqrt_diag.argtypes = [P, i64, P, P]
     lib.iq_status_string.restype = ctypes.c_char_p
@@ -230,7 +231,7 @@ def _blocks_ld(t: torch.Tensor, lead: tuple, nblk: int, B: int, name: str) -> in
 
 def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor,
                      picks: torch.Tensor | None = None, payload: torch.Tensor | None = None,
-                     flags: torch.Tensor | None = None, stream=None):
+                     flags: torch.Tensor | None = None, stream=None, objective: torch.Tensor | None = None):
     """Local-Hessian choice search over all 256-column blocks of w.
 
     w: bf16 [rows, cols] with hess fp32 [cols/256, 256, 256], or a stack of experts
@@ -239,6 +240,8 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     cand: uint8 [C, (experts,) rows, cols/256, B], the every-choice payloads (C = CHOICES[fmt]).
     w, cand and payload may be views (say one 256-column block of a wider weight and its slices):
     rows need only be evenly spaced, each block contiguous.
+    objective: optional contiguous fp32 [(experts,) rows, cols/256], filled with each row-block's
+    final Delta^T H Delta.
     Returns (picks uint8 [(experts,) rows, cols/256, G] contiguous, payload uint8
     [(experts,) rows, cols/256, B]).
     """
@@ -268,10 +271,13 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     if payload is None:
         payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=w.device)
     payload_ld = _blocks_ld(payload, lead, nblk, B, "payload")
+    if objective is not None and (objective.dtype != torch.float32 or tuple(objective.shape) != lead + (nblk,)
+                                  or not objective.is_contiguous() or not objective.is_cuda):
+        raise IQError(f"objective must be a contiguous float32 CUDA tensor of shape {lead + (nblk,)}")
     _check(lib.iq_choice_search(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(-2), hess.data_ptr(),
                                 rows_e, cand.data_ptr(), cand_ld, cand.stride(0), picks.data_ptr(),
-                                payload.data_ptr(), payload_ld, None if flags is None else flags.data_ptr(),
-                                _stream(stream)))
+                                payload.data_ptr(), payload_ld, None if objective is None else objective.data_ptr(),
+                                None if flags is None else flags.data_ptr(), _stream(stream)))
     return picks, payload
 
 

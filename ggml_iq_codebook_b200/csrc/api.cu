@@ -138,7 +138,7 @@ iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks
 iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows, int64_t nblk,
                            int64_t ldw, const float* hess, int64_t rows_per_hess, const uint8_t* cand, int64_t cand_ld,
                            int64_t cand_choice_stride, uint8_t* picks, uint8_t* payload,
-                           int64_t payload_ld, uint32_t* flags, cudaStream_t stream) {
+                           int64_t payload_ld, float* objective, uint32_t* flags, cudaStream_t stream) {
     iq_status st = check_desc(desc);
     if (st != IQ_OK) return st;
     if (w == nullptr || hess == nullptr || cand == nullptr || picks == nullptr || payload == nullptr)
@@ -165,6 +165,7 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     p.picks = picks;
     p.payload = payload;
     p.payload_ld = payload_ld;
+    p.objective = objective;
     p.flags = flags;
     p.grid = desc->grid;
     return launched(iqk::launch_choice_search(desc->fmt, p, sms, stream));

@@ -477,6 +477,20 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         }
     }
 
+    __syncthreads();  // every gradient update has landed
+
+    // ---- the final objective Delta^T H Delta = sum_i cur_i grad_i: lane c sums columns
+    // 16c .. 16c + 15 by a pairwise tree, then the butterfly joins the 16 lanes pairwise
+    if (p.objective != nullptr && active) {
+        float pr[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pr[j] = __fmul_rn(cur[16 * c + j], grad[16 * c + j]);
+        float t = tree_sum<16>(pr);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) t = __fadd_rn(t, __shfl_xor_sync(hmask, t, o));
+        if (c == 0) p.objective[row * p.nblk + blk] = t;
+    }
+
     // ---- step 4: picks and the payload assembled from the picked candidates
     if (active) {
         __syncwarp(hmask);

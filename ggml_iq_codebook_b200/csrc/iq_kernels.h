@@ -41,6 +41,7 @@ struct ChoiceParams {
     uint8_t* picks;
     uint8_t* payload;
     int64_t payload_ld;
+    float* objective;  // nullptr, or [rows][nblk]: the final Delta^T H Delta
     uint32_t* flags;
     const int8_t* grid;
 };

@@ -180,6 +180,8 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
  *   payload: the final payload, block (r, b) at payload + (r * payload_ld + b) * B: each choice
  *     group's fields copied from its picked candidate, d from candidate 0 (the encode under the
  *     picks, PR #3157).
+ *   objective: NULL, or fp32 [rows][nblk]: the final Delta^T H Delta of each row and block, as
+ *     sum_i Delta_i grad_i over the search's final gradient (a pairwise tree over the columns).
  * Steps per (row, block): Delta(c) = x - decode(cand c); each group takes its best choice under
  * its own H_gg; grad = H Delta; two sweeps over the groups in order, each taking the choice with
  * the least gain 2 u^T grad_g + u^T H_gg u (u = Delta_g(c) - Delta_g(cur)) iff that gain < 0,
@@ -188,7 +190,7 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
 iq_status iq_choice_search(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t nblk,
                            int64_t ldw, const float *hess, int64_t rows_per_hess, const uint8_t *cand,
                            int64_t cand_ld, int64_t cand_choice_stride, uint8_t *picks, uint8_t *payload,
-                           int64_t payload_ld, uint32_t *flags, cudaStream_t stream);
+                           int64_t payload_ld, float *objective, uint32_t *flags, cudaStream_t stream);
 
 /*
  * out[b * 256 + i] = sqrtf(hess[b][i][i]) for b < nblk: the search importance the local-Hessian

@@ -254,12 +254,14 @@ def test_local_hessian_pipeline_on_gpu_matches_oracle(dev, descs, grids, anchors
     imp = oracle.sqrt_diag(hess.numpy())
     assert np.array_equal(imp_d.cpu().numpy(), imp)
     cand_d = iq.iq_encode(descs[fmt], w.to(dev), imp_d, every_choice=True)
-    picks, pay = iq.iq_choice_search(descs[fmt], w.to(dev), hd, cand_d)
+    obj = torch.empty((rows, nblk), dtype=torch.float32, device=dev)
+    picks, pay = iq.iq_choice_search(descs[fmt], w.to(dev), hd, cand_d, objective=obj)
     cand, _ = oracle.encode(fmt, grids[fmt], anchors[fmt], w, importance=imp, every_choice=True)
-    want_p, want_pay = oracle.choice_search(fmt, grids[fmt], w, hess.numpy(), cand)
+    want_p, want_pay, want_obj = oracle.choice_search(fmt, grids[fmt], w, hess.numpy(), cand, objective=True)
     assert np.array_equal(cand_d.cpu().numpy(), cand)
     assert np.array_equal(picks.cpu().numpy(), want_p)
     assert np.array_equal(pay.cpu().numpy(), want_pay)
+    assert np.array_equal(obj.cpu().numpy().view(np.uint32), want_obj.view(np.uint32))  # fp32 bits
     # the final payload is the encode under the picks
     fixed = iq.iq_encode(descs[fmt], w.to(dev), imp_d, choices=picks.contiguous())
     assert torch.equal(fixed, pay)

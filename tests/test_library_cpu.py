@@ -90,14 +90,14 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert lib.iq_decode(ctypes.byref(d), W, 0, 1, W, None) == 2
     assert lib.iq_decode(ctypes.byref(d), W, 4, 7, W, None) == 1
     assert lib.iq_decode(ctypes.byref(d), None, 4, 1, W, None) == 1
-    assert lib.iq_choice_search(ctypes.byref(d), W, 0, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None) == 2
-    assert lib.iq_choice_search(ctypes.byref(d), W, 4, 2, 256, W, 0, W, 2, 0, W, W, 2, None, None) == 1
-    assert lib.iq_choice_search(ctypes.byref(d), W, 6, 1, 256, W, 4, W, 1, 0, W, W, 1, None, None) == 2  # 4 !| 6
+    assert lib.iq_choice_search(ctypes.byref(d), W, 0, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None, None) == 2
+    assert lib.iq_choice_search(ctypes.byref(d), W, 4, 2, 256, W, 0, W, 2, 0, W, W, 2, None, None, None) == 1
+    assert lib.iq_choice_search(ctypes.byref(d), W, 6, 1, 256, W, 4, W, 1, 0, W, W, 1, None, None, None) == 2  # 4 !| 6
     # IQ1_M: any anchor (it is derived per block)
     m = _desc(fmt=3, anchor=float("nan"))
     assert E(ctypes.byref(m), W, 0, 1, 512, 384, 384, 0, None, 0, None, None, 0, 0, W, None, None) == 2
-    assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, 3, W, 1, 0, W, W, 1, None, None) == 2  # 3 !| 4
+    assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, 3, W, 1, 0, W, W, 1, None, None, None) == 2  # 3 !| 4
     s2 = _desc(fmt=4, entries=1024, anchor=0.9)
-    assert lib.iq_choice_search(ctypes.byref(s2), W, 0, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None) == 2
+    assert lib.iq_choice_search(ctypes.byref(s2), W, 0, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None, None) == 2
     assert lib.iq_sqrt_diag(None, 1, W, None) == 1
     assert lib.iq_sqrt_diag(W, 0, W, None) == 2
