@@ -2,8 +2,9 @@
 
 A plain, slow C restatement (``iq_oracle.c``) of the IQ1_S / IQ1_M / IQ2_XS / IQ2_S encoder and
 decoder, and the local-Hessian choice search (all four formats), with this thin ctypes wrapper.
-It is the yardstick the CUDA library is checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import it; the library never does, and the two share no code.
+It is the yardstick the CUDA library is checked against. Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import it; the library
+never does, and the two share no code.
 
 Functions whose parity rests on invariants only (no value fixed by the pages or by a closed form)
 are marked "parity unpinned" in their docstrings.
