@@ -554,3 +554,37 @@ def test_iq2xs_lowest_index_wins_on_equal_error(grids, anchors):
             assert idx[grp] == ties.min(), grp
             tied += len(ties) >= 2
     assert tied >= 8
+
+
+# ------------------------------------------------------------------------------ joint enumeration
+
+def test_iq1s_joint_enumeration_on_a_reduced_grid(anchors):
+    """A 2048-entry grid holding only 16 distinct rows (each repeated) lets fp64 enumerate every
+    (choice, entry of each of the 4 groups) of a whole 32-weight sub-block jointly: 16 x 16^4
+    candidates. The oracle's separable search must reach that joint minimum."""
+    rng = np.random.default_rng(161)
+    rows16 = np.stack([rng.integers(-1, 2, 8) for _ in range(16)]).astype(np.int8)
+    grid = np.tile(rows16, (128, 1))                      # entry q is row q % 16
+    w, imp = _case(1, 256, 162)
+    p, f = oracle.encode("iq1_s", grid, anchors["iq1_s"], w, importance=imp)
+    assert f == 0
+    x, wi = w.double().numpy()[0], imp.double().numpy()
+    d, ls, neg, idx = iq1s_fields(p[0, 0])
+    for k in range(2):                                    # two sub-blocks, enumerated jointly
+        xs, ws = x[32 * k:32 * k + 32].reshape(4, 8), wi[32 * k:32 * k + 32].reshape(4, 8)
+        best = np.inf
+        for c in range(16):
+            s = d * (2 * (c & 7) + 1)
+            delta = -0.125 if c >= 8 else 0.125
+            xhat = s * (rows16.astype(np.float64) + delta)                     # [16, 8]
+            e = ((xs[:, None, :] - xhat[None]) ** 2 * ws[:, None, :]).sum(-1)  # [4 groups, 16]
+            joint = (e[0][:, None, None, None] + e[1][None, :, None, None]
+                     + e[2][None, None, :, None] + e[3][None, None, None, :])  # all 16^4 combinations
+            best = min(best, joint.min())
+        c = ls[k] + 8 * neg[k]
+        s = d * (2 * (c & 7) + 1)
+        delta = -0.125 if c >= 8 else 0.125
+        got = sum(float(((xs[i] - s * (grid[idx[4 * k + i]] + delta)) ** 2 * ws[i]).sum()) for i in range(4))
+        scale = float((ws * xs ** 2).sum())
+        assert got <= best + 2e-5 * scale, (k, got, best)
+        assert all(idx[4 * k + i] < 16 for i in range(4))  # ties resolve to the first copy of a row
