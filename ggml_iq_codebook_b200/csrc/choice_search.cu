@@ -19,21 +19,21 @@
 // Experts: a stack of weights sharing a row layout runs in the same launch, row r taking Hessian
 // set r / rows_per_hess (PR #3218's reason for one launch: thousands of small expert weights).
 //
-// Design (B200): one CTA = 16 (IQ2_XS, IQ2_S) or 8 (IQ1_S) rows of one block, a half-warp per row and
-// one lane per choice. The
-// rows run the group steps in lockstep, so each step stages one panel of H (the group's W rows,
-// W x 256 fp32) in shared memory once for all rows, double-buffered with cp.async so the next
-// panel streams in while this one is used; H is read from L2 three times per CTA (step 2 fused
+// Design (B200): one CTA = 16 rows (8 for IQ1_S) of one block, a half-warp per row and one lane per
+// choice. The rows run the group steps in lockstep, so each step stages one panel of H (the group's
+// W rows, W x 256 fp32) in shared memory once for all rows, double-buffered with cp.async so the
+// next panel streams in while this one is used; H is read from L2 three times per CTA (step 2 fused
 // with the initial gradient, then one pass per sweep). A lane decodes its own candidate's group
-// straight into registers and keeps all W accumulators of H_gg u: W independent fma chains fed
-// by broadcast 16-byte panel reads. Its two trees are local, and the only cross-lane step is a
-// 4-level argmin over the half-warp; the winning lane writes cur and u from its registers. The
-// gradient work (the initial H Delta, and after every sweep step the updates of the rows that
-// switched) is done by all threads together: the initial H Delta as 4-row x 4-column register
-// tiles (per k one 16-byte read of the rows' values and one of H, then 16 fmas); after a sweep
-// step, by column when few rows switched (each thread holding its H column and walking only those
-// rows), else by the same tiles. The grid is staged as
-// 16-bit element codes, so decoding needs no int-to-float conversions.
+// straight into registers and keeps all W accumulators of H_gg u: W independent fma chains fed by
+// broadcast 16-byte panel reads. Its two trees are local, and the only cross-lane step is a 4-level
+// argmin over the half-warp; the winning lane writes cur and u from its registers. The gradient
+// work (the initial H Delta, and after every sweep step the updates of the rows that switched) is
+// done by all threads together: the initial H Delta as 4-row x 4-column register tiles (per k one
+// 16-byte read of the rows' values and one of H, then 16 fmas); after a sweep step, by column when
+// few rows switched (each thread holding its H column and walking only those rows), else by the
+// same tiles. The grid is staged as 16-bit element codes, so decoding needs no int-to-float
+// conversions. On request each row's final Delta^T H Delta is reported as sum_i cur_i grad_i (a
+// pairwise tree over the 256 columns).
 #include "iq_device.cuh"
 #include "iq_kernels.h"
 

@@ -12,7 +12,8 @@
 //              + (sum over its high-nibble bits, ascending from 0);  W = S(w, all), Tall = S(T, all)
 //   per entry  P/N = positions of +1/-1;  A = S(w,P) + S(w,N);  R = S(w,P) - S(w,N);
 //              C = S(T,P) - S(T,N)
-//   per choice A_d = fma(d^2, W, fma(2 d, R, A));  C_d = fma(d, Tall, C);  m = fma(s, A_d, C_d)
+//   per choice A_delta = fma(delta^2, W, fma(2 delta, R, A));  C_delta = fma(delta, Tall, C);
+//              m = fma(s, A_delta, C_delta)
 //   per (group, c)     argmin_q m (lowest q on ties), e = s * m_min
 //   per (sub-block, c) E = (e0 + e1) + (e2 + e3);  choice = argmin_c E (lowest c on ties)
 //
@@ -28,8 +29,10 @@
 // 16 low and 16 high nibble values, 8 KiB per warp, conflict-free rows). The argmin keeps only
 // running minima (fminf) in registers plus the chunk of K entries where each choice's minimum
 // first appeared (two candidates fold into one three-input min); the winning entry index is
-// recovered afterwards by rescanning that one chunk with the identical arithmetic. Persistent CTAs walk the blocks with a static stride: every
-// block costs the same, so no work queue (and no scratch memory) is needed.
+// recovered afterwards by rescanning that one chunk with the identical arithmetic. Persistent
+// CTAs walk the blocks with a static stride: every block costs the same, so no work queue (and
+// no scratch memory) is needed. Weights arrive as bf16 (its own instantiation), f16 or fp32, all
+// converted exactly; d is predicted from amax or given per block (static scales, PR #3197).
 #include "iq_device.cuh"
 #include "iq_kernels.h"
 

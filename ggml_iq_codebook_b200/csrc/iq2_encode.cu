@@ -18,9 +18,9 @@
 // 82-byte block holds d, the low index bytes, the sign bytes, the 2-bit high index fields (group
 // g at shift 2 (g % 4) of byte 66 + g/4) and the scale nibbles at bytes 74..81.
 //
-// Kernel design (B200): one warp per block, one lane per group; the 512-entry loop is warp-uniform
-// and reads each entry's 8 magnitudes and 8 squares (64 B) with broadcast 16-byte shared-memory
-// loads. Argmin bookkeeping as in the IQ1_S kernel: running minima, chunk of first appearance,
+// Kernel design (B200): one warp per block, one lane per group; the entry loop (512 entries for
+// IQ2_XS, 1024 for IQ2_S) is warp-uniform and reads each entry's 8 magnitudes and 8 squares
+// (64 B) with broadcast 16-byte shared-memory loads. Argmin bookkeeping as in the IQ1_S kernel: running minima, chunk of first appearance,
 // one-chunk rescan for the index; the rescans, whose entries differ from lane to lane, read a
 // packed 8-byte copy of the grid instead of the 64-byte float rows.
 #include "iq_device.cuh"

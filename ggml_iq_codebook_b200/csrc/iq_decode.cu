@@ -14,11 +14,12 @@
 // output is its round-to-nearest-even. Each block decodes independently, so the output does not
 // depend on how a caller chunks the blocks.
 //
-// Design: persistent CTAs walk tiles of 256 blocks. A tile's payload bytes (12.5 / 18.5 KiB)
+// Design: persistent CTAs walk tiles of 256 blocks. A tile's payload bytes (12.5, 14, 18.5 or
+// 20.5 KiB for IQ1_S, IQ1_M, IQ2_XS, IQ2_S)
 // stream into shared memory with 16-byte cp.async copies, double-buffered, so the next tile's
 // reads are in flight while this one is decoded and no warp waits on its own small global loads.
 // A half-warp decodes one block, two adjacent 8-weight groups per lane, reading its fields from
-// the staged bytes; the grid is staged once per CTA as 16-bit element codes (4 KiB / 1 KiB), and
+// the staged bytes; the grid is staged once per CTA as 16-bit element codes (4, 1 or 2 KiB), and
 // outputs are picked from a lane's precomputed products (no int-to-float conversions, which
 // throttle the MIO queue). Each lane writes its 16 outputs with 32-byte streaming stores
 // (st.global.v8): one for bf16, two for fp32.
