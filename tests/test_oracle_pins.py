@@ -588,3 +588,29 @@ def test_iq1s_joint_enumeration_on_a_reduced_grid(anchors):
         scale = float((ws * xs ** 2).sum())
         assert got <= best + 2e-5 * scale, (k, got, best)
         assert all(idx[4 * k + i] < 16 for i in range(4))  # ties resolve to the first copy of a row
+
+
+def test_iq2xs_joint_enumeration_on_a_reduced_grid(anchors):
+    """512 entries made of 16 distinct magnitude rows: fp64 enumerates every (ls, entry, entry) of
+    a 16-weight sub-block jointly (16 x 16^2) under the signs the encoder fixed; the oracle must
+    reach that minimum, and repeated rows resolve to their first copy."""
+    rng = np.random.default_rng(171)
+    rows16 = np.stack([rng.choice([1, 3, 5, 7], 8) for _ in range(16)]).astype(np.int8)
+    grid = np.tile(rows16, (32, 1))
+    w, imp = _case(1, 256, 172, std=0.015)
+    p, f = oracle.encode("iq2_xs", grid, anchors["iq2_xs"], w, importance=imp)
+    assert f == 0
+    x, wi = w.double().numpy()[0], imp.double().numpy()
+    d, ls, idx, s7 = iq2xs_fields(p[0, 0])
+    signs = iq2xs_signs(s7)
+    for k in range(4):
+        xs, ws = x[16 * k:16 * k + 16].reshape(2, 8), wi[16 * k:16 * k + 16].reshape(2, 8)
+        best = np.inf
+        for l in range(16):
+            s = d * (2 * l + 1)
+            e = [((xs[i][None] - s * rows16 * signs[2 * k + i][None]) ** 2 * ws[i][None]).sum(-1) for i in range(2)]
+            best = min(best, (e[0][:, None] + e[1][None, :]).min())
+        s = d * (2 * ls[k] + 1)
+        got = sum(float(((xs[i] - s * grid[idx[2 * k + i]] * signs[2 * k + i]) ** 2 * ws[i]).sum()) for i in range(2))
+        assert got <= best + 2e-5 * float((ws * xs ** 2).sum()), (k, got, best)
+        assert idx[2 * k] < 16 and idx[2 * k + 1] < 16
