@@ -14,7 +14,9 @@
 // updates grad_i by an fma chain over the group's k. NaN and +inf scores never win.
 //
 // Formats: IQ1_S (8 groups of 32 columns), IQ2_XS and IQ2_S (16 groups of 16 columns), 16 choices;
-// IQ1_M (16 groups of 16 columns, 8 choices: the other 8 lanes of a row never win).
+// IQ1_M (16 groups of 16 columns, 8 choices). With 8 choices two lanes share a candidate and each
+// forms half of the group's H_gg u columns and half of each score's products; a 16-wide pairwise
+// tree ends by adding its two 8-wide subtrees, so the halves join with one shuffle and one add.
 //
 // Experts: a stack of weights sharing a row layout runs in the same launch, row r taking Hessian
 // set r / rows_per_hess (PR #3218's reason for one launch: thousands of small expert weights).
@@ -163,6 +165,8 @@ struct Cfg {
                                                    : kIq2xsBytes;
     static constexpr int E = FMT == IQ_FMT_IQ2_XS ? kIq2xsEntries : FMT == IQ_FMT_IQ2_S ? kIq2sEntries : kIq1sEntries;
     static constexpr int NC = FMT == IQ_FMT_IQ1_M ? kIq1mChoices : kChoices;  // candidates per row
+    static constexpr int SPLIT = kChoices / NC;                 // lanes per candidate
+    static constexpr int WO = W / SPLIT;                        // group columns per lane
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
     // shared memory layout (bytes)
     static constexpr int oHp = 0;                                 // float [2][W][256], double buffer
@@ -207,29 +211,43 @@ __device__ __forceinline__ void half_argmin(float v, int c, unsigned mask, float
     cbest = c;
 }
 
-// v[i] = sum over k < W (fma chain, k ascending) of Hp[k][col0 + i] * a[k], all W columns.
+// v[i] = sum over k < W (fma chain, k ascending) of Hp[k][col0 + i] * a[k], for NO columns.
 // The next panel row is loaded while the current one is used (software pipelining).
-template <int W>
-__device__ __forceinline__ void group_matvec(const float* Hp, int col0, const float a[W], float v[W]) {
-    float h[W], hn[W];
-    load_vec<W>(Hp + col0, h);
-    load_vec<W>(Hp + kBlock + col0, hn);
+template <int W, int NO>
+__device__ __forceinline__ void group_matvec(const float* Hp, int col0, const float a[W], float v[NO]) {
+    float h[NO], hn[NO];
+    load_vec<NO>(Hp + col0, h);
+    load_vec<NO>(Hp + kBlock + col0, hn);
 #pragma unroll
-    for (int i = 0; i < W; ++i) v[i] = __fmul_rn(h[i], a[0]);
+    for (int i = 0; i < NO; ++i) v[i] = __fmul_rn(h[i], a[0]);
 #pragma unroll
     for (int k = 1; k < W; ++k) {
 #pragma unroll
-        for (int i = 0; i < W; ++i) h[i] = hn[i];
-        if (k + 1 < W) load_vec<W>(Hp + (k + 1) * kBlock + col0, hn);
+        for (int i = 0; i < NO; ++i) h[i] = hn[i];
+        if (k + 1 < W) load_vec<NO>(Hp + (k + 1) * kBlock + col0, hn);
 #pragma unroll
-        for (int i = 0; i < W; ++i) v[i] = __fmaf_rn(h[i], a[k], v[i]);
+        for (int i = 0; i < NO; ++i) v[i] = __fmaf_rn(h[i], a[k], v[i]);
     }
+}
+
+// This lane's half of a group vector (register indices stay static), or all of it.
+template <int W, int WO>
+__device__ __forceinline__ void lane_part(const float a[W], int part, float out[WO]) {
+#pragma unroll
+    for (int i = 0; i < WO; ++i) out[i] = (WO < W && part) ? a[WO + i] : a[i];
+}
+
+// Joins the two halves' tree sums (lanes c and c + NC) when a candidate spans two lanes.
+template <int SPLIT, int NC>
+__device__ __forceinline__ float join_parts(float t, unsigned mask) {
+    return SPLIT == 1 ? t : __fadd_rn(t, __shfl_xor_sync(mask, t, NC));
 }
 
 template <int FMT>
 __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const ChoiceParams p) {
     using C = Cfg<FMT>;
-    constexpr int W = C::W, G = C::G, kRows = C::R, kThreads = C::T;
+    constexpr int W = C::W, G = C::G, kRows = C::R, kThreads = C::T, WO = C::WO;
+    static_assert(C::SPLIT * C::NC == kChoices && (W & (W - 1)) == 0, "halves join as the tree's last level");
     static_assert(kThreads == C::RG * 64, "gradient tiles: 4 rows x 4 columns per thread");
     static_assert(2 * W * kRows <= kBlock * kRows, "u buffers fit in the curT area");
     extern __shared__ __align__(16) char smem[];
@@ -248,6 +266,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     const int64_t expert = rem / tiles_e;
     const int64_t tile_row0 = (rem - expert * tiles_e) * kRows;
     const int tid = threadIdx.x, hr = tid >> 4, c = tid & 15;
+    const int ch = c % C::NC, part = c / C::NC;  // this lane's candidate, and its half of the columns
     const unsigned hmask = 0xFFFFu << (16 * (hr & 1));  // this half-warp's lanes within the warp
     const int64_t row = expert * p.rows_per_hess + tile_row0 + hr;
     const bool active = tile_row0 + hr < p.rows_per_hess;
@@ -309,7 +328,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
 #pragma unroll
         for (int t = 0; t < W / 8; ++t) {
             float xh[8], xv[8];
-            decode8<FMT>(cand + c * C::B, sgrid, g, (g * W + 8 * t) >> 3, xh);
+            decode8<FMT>(cand + ch * C::B, sgrid, g, (g * W + 8 * t) >> 3, xh);
             unpack8_bf16(reinterpret_cast<const uint4*>(xb)[(g * W) / 8 + t], xv);
 #pragma unroll
             for (int j = 0; j < 8; ++j) dl[8 * t + j] = __fsub_rn(xv[j], xh[j]);
@@ -334,12 +353,17 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         prefetch(g + 1);
         const float* Hp = panel(g);
         if (active) {
-            float dl[W], v[W];
+            float dl[W], v[WO];
             delta_of(g, dl);
-            group_matvec<W>(Hp, g * W, dl, v);
+            group_matvec<W, WO>(Hp, g * W + part * WO, dl, v);
+            {
+                float dp[WO];
+                lane_part<W, WO>(dl, part, dp);
 #pragma unroll
-            for (int i = 0; i < W; ++i) v[i] = __fmul_rn(dl[i], v[i]);
-            const float score = c < C::NC ? tree_sum<W>(v) : INFINITY;
+                for (int i = 0; i < WO; ++i) v[i] = __fmul_rn(dp[i], v[i]);
+            }
+            const float t = join_parts<C::SPLIT, C::NC>(tree_sum<WO>(v), hmask);
+            const float score = c < C::NC ? t : INFINITY;
             float best;
             int cstar;
             half_argmin(score, c, hmask, best, cstar);
@@ -389,7 +413,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         const float* Hp = panel(step);
         int switched = 0;
         if (active) {
-            float dl[W], u[W], v[W];
+            float dl[W], u[W], v[WO];
             delta_of(g, dl);
             {
                 float cgv[W];
@@ -397,17 +421,19 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
 #pragma unroll
                 for (int i = 0; i < W; ++i) u[i] = __fsub_rn(dl[i], cgv[i]);
             }
-            group_matvec<W>(Hp, g * W, u, v);
+            group_matvec<W, WO>(Hp, g * W + part * WO, u, v);
             float gain;
             {
-                float gq[W], p1[W];
-                load_vec<W>(grad + g * W, gq);
+                float gq[WO], p1[WO], up[WO];
+                load_vec<WO>(grad + g * W + part * WO, gq);
+                lane_part<W, WO>(u, part, up);
 #pragma unroll
-                for (int i = 0; i < W; ++i) {
-                    p1[i] = __fmul_rn(u[i], gq[i]);
-                    v[i] = __fmul_rn(u[i], v[i]);
+                for (int i = 0; i < WO; ++i) {
+                    p1[i] = __fmul_rn(up[i], gq[i]);
+                    v[i] = __fmul_rn(up[i], v[i]);
                 }
-                const float t1 = tree_sum<W>(p1), t2 = tree_sum<W>(v);
+                const float t1 = join_parts<C::SPLIT, C::NC>(tree_sum<WO>(p1), hmask);
+                const float t2 = join_parts<C::SPLIT, C::NC>(tree_sum<WO>(v), hmask);
                 gain = c < C::NC ? __fmaf_rn(2.0f, t1, t2) : INFINITY;
             }
             float best;
