@@ -27,6 +27,7 @@ FMT = {"iq1_s": 1, "iq2_xs": 2, "iq1_m": 3, "iq2_s": 4}
 BLOCK_BYTES = {"iq1_s": 50, "iq2_xs": 74, "iq1_m": 56, "iq2_s": 82}
 CHOICE_GROUPS = {"iq1_s": 8, "iq2_xs": 16, "iq1_m": 16, "iq2_s": 16}
 CHOICES = {"iq1_s": 16, "iq2_xs": 16, "iq1_m": 8, "iq2_s": 16}
+CS_IQ2XS_G8 = 5  # choice-search layout code: IQ2_XS candidates, 32 groups of 8 columns, ls 8..15
 NUM_CHOICES = 16
 
 FLAG_NONFINITE = 1
@@ -217,6 +218,41 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     out = [picks.reshape(lead + (nblk, G)), payload.reshape(lead + (nblk, B))]
     if trace:
         out.append(tr.reshape(lead + (nblk, 3, G)))
+    if objective:
+        out.append(obj.reshape(lead + (nblk,)))
+    return tuple(out)
+
+
+def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False,
+                     objective=False):
+    """The local-Hessian choice search with eight candidates per 8-weight group: 32 groups of 8
+    columns per block, each choosing among the IQ2_XS every-choice decodes for ls = 8..15.
+
+    w and hess as in choice_search; cand: the 16-choice IQ2_XS every-choice encode
+    [16, (experts,) rows, nblk, 74], of which choices 8..15 are read. Returns (picks,) with picks
+    [(experts,) rows, nblk, 32] holding the chosen ls (8..15); with trace, also the picks after
+    step 2 and after each sweep [(experts,) rows, nblk, 3, 32]; with objective (last), each
+    row-block's final Delta^T H Delta. No payload layout stores a scale per 8 weights, so none
+    is assembled.
+    """
+    wb = _bf16_bits(w)
+    lead = wb.shape[:-1]
+    cols = wb.shape[-1]
+    wb = wb.reshape(-1, cols)
+    rows = wb.shape[0]
+    nexp = wb.shape[0] // lead[-1] if len(lead) == 2 else 1
+    nblk = cols // 256
+    hess = np.ascontiguousarray(hess, dtype=np.float32).reshape(nexp, nblk, 256, 256)
+    cand = np.ascontiguousarray(cand, dtype=np.uint8).reshape(16, rows, nblk, 74)
+    picks = np.zeros((rows, nblk, 32), dtype=np.uint8)
+    tr = np.zeros((rows, nblk, 3, 32), dtype=np.uint8) if trace else None
+    obj = np.zeros((rows, nblk), dtype=np.float32) if objective else None
+    _load().orc_choice_search(CS_IQ2XS_G8, _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
+                              rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
+                              None, _ptr(tr), _ptr(obj))
+    out = [picks.reshape(lead + (nblk, 32))]
+    if trace:
+        out.append(tr.reshape(lead + (nblk, 3, 32)))
     if objective:
         out.append(obj.reshape(lead + (nblk,)))
     return tuple(out)
