@@ -49,7 +49,8 @@ L2_FLUSH_BYTES = 256 << 20
 #     own-block scores G x C x (W^2 + 2W - 1), gradient 256 x 256, two sweeps of
 #     G x C x (W^2 + 5W - 1) gains; gradient updates after a switch are data dependent and not
 #     counted. IQ2_XS and IQ2_S (G = C = 16): 310,528 ops; IQ1_S (G = 8, C = 16): 507,520 ops;
-#     IQ1_M (G = 16, C = 8): 188,032 ops.
+#     IQ1_M (G = 16, C = 8): 188,032 ops; eight candidates per 8-weight group (G = 32, C = 8):
+#     138,496 ops.
 #   IQ1_M runs IQ1_S's search (same 2048 x 16 candidates per group): 2,949,120 ops per block.
 #   IQ2_S runs IQ2_XS's per-entry work over 1024 entries: 32 x 1024 x 48 = 1,572,864 per block.
 OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120, "iq2_s": 1_572_864}
@@ -185,6 +186,9 @@ WORKLOADS = {
     "choice_iq1s_4096x4096": ("iq1_s", [4096, 4096], _choice_text("iq1_s", "4096x4096", False)),
     "choice_iq1m_4096x4096": ("iq1_m", [4096, 4096], _choice_text("iq1_m", "4096x4096", False)),
     "choice_iq2xs_moe_16x1536x4096": ("iq2_xs", [16, 1536, 4096], _choice_text("iq2_xs", "16x1536x4096", True)),
+    "choice_iq2xs_g8_4096x4096": ("iq2_xs", [4096, 4096], _choice_text("iq2_xs", "4096x4096", False)
+                                  + ", eight candidates (ls 8..15) per 8-weight group over 32 groups of 8 "
+                                  "columns, picks only"),
     "choice_iq2xs_4096x4096_per_block": ("iq2_xs", [4096, 4096], _choice_text("iq2_xs", "4096x4096", False)
                                          + ", the search as one call per 256-column block (16 calls)"),
     "iq1s_decode_1m_blocks": ("iq1_s", [4096, 4096], "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 "
@@ -198,6 +202,7 @@ class Workload:
     def __init__(self, name: str, dev, peaks):
         self.name, self.dev, self.peaks = name, dev, peaks
         self.per_block = False
+        self.g8 = "_g8_" in name  # eight candidates per 8-weight group: picks only
         g1 = torch.from_numpy(synth.iq1s_grid()).to(dev)
         g2 = torch.from_numpy(synth.iq2xs_grid()).to(dev)
         g3 = torch.from_numpy(synth.iq2s_grid()).to(dev)
@@ -263,7 +268,7 @@ class Workload:
         nblk = cols // 256
         nexp = lead[0] if len(lead) == 2 else 1
         self.imp = torch.empty((nexp, cols) if len(lead) == 2 else (cols,), dtype=torch.float32, device=self.dev)
-        B, G = iq.BLOCK_BYTES[fmt], iq.CHOICE_GROUPS[fmt]
+        B, G = iq.BLOCK_BYTES[fmt], (32 if self.g8 else iq.CHOICE_GROUPS[fmt])
         self.cand = torch.empty((iq.CHOICES[fmt],) + lead + (nblk, B), dtype=torch.uint8, device=self.dev)
         self.picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=self.dev)
         self.picks_b = torch.empty((nblk,) + lead + (1, G), dtype=torch.uint8, device=self.dev)
@@ -273,7 +278,7 @@ class Workload:
         self.launches_per_step = 3
         self.text = text
         self.dominant = "choice_search_kernel"
-        self.ops_per_launch = self.nblocks * choice_ops_per_row_block(G, iq.CHOICES[fmt])
+        self.ops_per_launch = self.nblocks * choice_ops_per_row_block(G, 8 if self.g8 else iq.CHOICES[fmt])
         iq.iq_sqrt_diag(self.hess, out=self.imp)
         iq.iq_encode(self.desc[fmt], self.w, self.imp, every_choice=True, out=self.cand)
 
@@ -303,6 +308,8 @@ class Workload:
                     iq.iq_choice_search(d, self.w[:, 256 * b:256 * (b + 1)], self.hess[b:b + 1],
                                         self.cand[:, :, b:b + 1], picks=self.picks_b[b],
                                         payload=self.payload[:, b:b + 1])
+            elif self.g8:
+                iq.iq_choice_search_g8(d, self.w, self.hess, self.cand, picks=self.picks)
             else:
                 iq.iq_choice_search(d, self.w, self.hess, self.cand, picks=self.picks, payload=self.payload)
             if ev is not None:
@@ -329,7 +336,8 @@ class Workload:
             self.step()
             picks = self.picks_b if self.per_block else self.picks
             host["picks"].view(-1).copy_(picks.view(-1), non_blocking=True)
-            host["payload"].copy_(self.payload, non_blocking=True)
+            if not self.g8:
+                host["payload"].copy_(self.payload, non_blocking=True)
 
     def host_buffers(self):
         pin = lambda t: t.to("cpu").pin_memory()  # noqa: E731
@@ -346,7 +354,7 @@ class Workload:
             h = {"w": pin(self.w_host), "hess": pin(self.hess_host), "picks": pin(self.picks),
                  "payload": pin(self.payload)}
             h2d = self.w.numel() * 2 + self.hess.numel() * 4
-            d2h = self.picks.numel() + self.payload.numel()
+            d2h = self.picks.numel() + (0 if self.g8 else self.payload.numel())
         return h, h2d, d2h
 
 
@@ -394,7 +402,8 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
     if name.startswith("choice_"):
         cfmt = {"choice_iq2xs_4096x4096": "iq2_xs", "choice_iq2s_4096x4096": "iq2_s",
                 "choice_iq1s_4096x4096": "iq1_s", "choice_iq1m_4096x4096": "iq1_m",
-                "choice_iq2xs_moe_16x1536x4096": "iq2_xs", "choice_iq2xs_4096x4096_per_block": "iq2_xs"}[name]
+                "choice_iq2xs_moe_16x1536x4096": "iq2_xs", "choice_iq2xs_4096x4096_per_block": "iq2_xs",
+                "choice_iq2xs_g8_4096x4096": "iq2_xs"}[name]
         if "moe" in name:  # the sample is the first rows of expert 0, under its own Hessians
             wl = synth.workload_choice_moe()
             w, hess = wl["w"][0], wl["hess"][0].numpy()
@@ -407,7 +416,10 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
 
         def run(r):
             cand, _ = oracle.encode(cfmt, g, iq.DEFAULT_ANCHOR[cfmt], w[:r], importance=imp, every_choice=True)
-            oracle.choice_search(cfmt, g, w[:r], hess, cand)
+            if "_g8_" in name:
+                oracle.choice_search_g8(g, w[:r], hess, cand)
+            else:
+                oracle.choice_search(cfmt, g, w[:r], hess, cand)
         cols = w.shape[1]
     else:
         if name == "iq1s_moe_256x1536x4096":

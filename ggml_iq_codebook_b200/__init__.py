@@ -4,7 +4,8 @@ Thin ctypes marshalling over the C ABI in include/iq.h: torch tensors supply dev
 the current CUDA stream, every computation runs in the library's kernels. There is no CPU path:
 if the shared library is missing or the device is not an sm_100 part, calls raise.
 
-Functions keep the C names: iq_encode, iq_decode, iq_choice_search, iq_sqrt_diag.
+Functions keep the C names: iq_encode, iq_decode, iq_choice_search, iq_choice_search_g8,
+iq_sqrt_diag.
 """
 
 from __future__ import annotations
@@ -33,7 +34,7 @@ IQ_IN = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
 
 SYMBOLS = ("iq_block_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
-           "iq_choice_search", "iq_sqrt_diag", "iq_status_string", "iq_build_info")
+           "iq_choice_search", "iq_choice_search_g8", "iq_sqrt_diag", "iq_status_string", "iq_build_info")
 
 
 class IQError(RuntimeError):
@@ -71,6 +72,8 @@ def load_library(path: str = LIB_PATH):
     lib.iq_choice_search.restype = ctypes.c_int
     lib.iq_choice_search.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, i64, P, i64, i64, P, P, i64, P, P,
                                      P]
+    lib.iq_choice_search_g8.restype = ctypes.c_int
+    lib.iq_choice_search_g8.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, i64, P, i64, i64, P, P, P, P]
     lib.iq_sqrt_diag.restype = ctypes.c_int
     lib.iq_sqrt_diag.argtypes = [P, i64, P, P]
     lib.iq_status_string.restype = ctypes.c_char_p
@@ -229,6 +232,33 @@ def _blocks_ld(t: torch.Tensor, lead: tuple, nblk: int, B: int, name: str) -> in
     return t.stride(-3) // B
 
 
+def _choice_args(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor, nchoice: int):
+    """Checks shared by both choice searches: (fmt, lead, rows, rows per Hessian set, nblk, cand_ld)."""
+    fmt = _fmt_of(desc)
+    _need(w, torch.bfloat16, "w")
+    _need(hess, torch.float32, "hess")
+    _need(cand, torch.uint8, "cand")
+    if w.dim() not in (2, 3) or w.stride(-1) != 1:
+        raise IQError("w must be [rows, cols] or [experts, rows, cols] with a contiguous last dim")
+    lead, cols = tuple(w.shape[:-1]), w.shape[-1]
+    nexp, rows_e = (lead[0], lead[1]) if w.dim() == 3 else (1, lead[0])
+    if w.dim() == 3 and nexp > 1 and w.stride(0) != rows_e * w.stride(1):
+        raise IQError("the experts of w must be evenly spaced in the row dimension")
+    nblk = cols // 256
+    B = BLOCK_BYTES[fmt]
+    if not hess.is_contiguous() or hess.numel() != nexp * nblk * 256 * 256:
+        raise IQError("hess must be contiguous [(experts,) cols/256, 256, 256]")
+    if cand.dim() != len(lead) + 3 or cand.shape[0] != nchoice:
+        raise IQError(f"cand must be [{nchoice}, (experts,) rows, cols/256, {B}]")
+    return fmt, lead, nexp * rows_e, rows_e, nblk, _blocks_ld(cand, lead, nblk, B, "cand")
+
+
+def _objective_ok(objective, lead, nblk):
+    if objective is not None and (objective.dtype != torch.float32 or tuple(objective.shape) != lead + (nblk,)
+                                  or not objective.is_contiguous() or not objective.is_cuda):
+        raise IQError(f"objective must be a contiguous float32 CUDA tensor of shape {lead + (nblk,)}")
+
+
 def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor,
                      picks: torch.Tensor | None = None, payload: torch.Tensor | None = None,
                      flags: torch.Tensor | None = None, stream=None, objective: torch.Tensor | None = None):
@@ -246,24 +276,8 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     [(experts,) rows, cols/256, B]).
     """
     lib = load_library()
-    fmt = _fmt_of(desc)
-    _need(w, torch.bfloat16, "w")
-    _need(hess, torch.float32, "hess")
-    _need(cand, torch.uint8, "cand")
-    if w.dim() not in (2, 3) or w.stride(-1) != 1:
-        raise IQError("w must be [rows, cols] or [experts, rows, cols] with a contiguous last dim")
-    lead, cols = tuple(w.shape[:-1]), w.shape[-1]
-    nexp, rows_e = (lead[0], lead[1]) if w.dim() == 3 else (1, lead[0])
-    if w.dim() == 3 and nexp > 1 and w.stride(0) != rows_e * w.stride(1):
-        raise IQError("the experts of w must be evenly spaced in the row dimension")
-    rows = nexp * rows_e
-    nblk = cols // 256
+    fmt, lead, rows, rows_e, nblk, cand_ld = _choice_args(desc, w, hess, cand, CHOICES[_fmt_of(desc)])
     B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
-    if not hess.is_contiguous() or hess.numel() != nexp * nblk * 256 * 256:
-        raise IQError("hess must be contiguous [(experts,) cols/256, 256, 256]")
-    if cand.dim() != len(lead) + 3 or cand.shape[0] != CHOICES[fmt]:
-        raise IQError(f"cand must be [{CHOICES[fmt]}, (experts,) rows, cols/256, {B}]")
-    cand_ld = _blocks_ld(cand, lead, nblk, B, "cand")
     if picks is None:
         picks = torch.empty(lead + (nblk, G), dtype=torch.uint8, device=w.device)
     elif picks.dtype != torch.uint8 or tuple(picks.shape) != lead + (nblk, G) or not picks.is_contiguous():
@@ -271,14 +285,38 @@ def iq_choice_search(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: to
     if payload is None:
         payload = torch.empty(lead + (nblk, B), dtype=torch.uint8, device=w.device)
     payload_ld = _blocks_ld(payload, lead, nblk, B, "payload")
-    if objective is not None and (objective.dtype != torch.float32 or tuple(objective.shape) != lead + (nblk,)
-                                  or not objective.is_contiguous() or not objective.is_cuda):
-        raise IQError(f"objective must be a contiguous float32 CUDA tensor of shape {lead + (nblk,)}")
+    _objective_ok(objective, lead, nblk)
     _check(lib.iq_choice_search(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(-2), hess.data_ptr(),
                                 rows_e, cand.data_ptr(), cand_ld, cand.stride(0), picks.data_ptr(),
                                 payload.data_ptr(), payload_ld, None if objective is None else objective.data_ptr(),
                                 None if flags is None else flags.data_ptr(), _stream(stream)))
     return picks, payload
+
+
+def iq_choice_search_g8(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.Tensor,
+                        picks: torch.Tensor | None = None, flags: torch.Tensor | None = None, stream=None,
+                        objective: torch.Tensor | None = None) -> torch.Tensor:
+    """The choice search with eight candidates per 8-weight group (IQ2_XS only): 32 groups of 8
+    columns per block, each choosing among the every-choice decodes for ls = 8..15.
+
+    w, hess, objective as in iq_choice_search; cand: uint8 [16, (experts,) rows, cols/256, 74],
+    the IQ2_XS every-choice payloads (choices 8..15 are read). Returns picks uint8
+    [(experts,) rows, cols/256, 32] holding the chosen ls (8..15); no payload is written.
+    """
+    lib = load_library()
+    if _fmt_of(desc) != "iq2_xs":
+        raise IQError("iq_choice_search_g8 takes IQ2_XS candidates")
+    fmt, lead, rows, rows_e, nblk, cand_ld = _choice_args(desc, w, hess, cand, CHOICES["iq2_xs"])
+    if picks is None:
+        picks = torch.empty(lead + (nblk, 32), dtype=torch.uint8, device=w.device)
+    elif picks.dtype != torch.uint8 or tuple(picks.shape) != lead + (nblk, 32) or not picks.is_contiguous():
+        raise IQError(f"picks must be a contiguous uint8 tensor of shape {lead + (nblk, 32)}")
+    _objective_ok(objective, lead, nblk)
+    _check(lib.iq_choice_search_g8(ctypes.byref(desc), w.data_ptr(), rows, nblk, w.stride(-2), hess.data_ptr(),
+                                   rows_e, cand.data_ptr(), cand_ld, cand.stride(0), picks.data_ptr(),
+                                   None if objective is None else objective.data_ptr(),
+                                   None if flags is None else flags.data_ptr(), _stream(stream)))
+    return picks
 
 
 def iq_sqrt_diag(hess: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

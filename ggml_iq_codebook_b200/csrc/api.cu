@@ -171,6 +171,42 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     return launched(iqk::launch_choice_search(desc->fmt, p, sms, stream));
 }
 
+iq_status iq_choice_search_g8(const iq_desc* desc, const uint16_t* w, int64_t rows, int64_t nblk, int64_t ldw,
+                              const float* hess, int64_t rows_per_hess, const uint8_t* cand, int64_t cand_ld,
+                              int64_t cand_choice_stride, uint8_t* picks, float* objective, uint32_t* flags,
+                              cudaStream_t stream) {
+    iq_status st = check_desc(desc);
+    if (st != IQ_OK) return st;
+    if (desc->fmt != IQ_FMT_IQ2_XS) return IQ_EUNSUPPORTED;
+    if (w == nullptr || hess == nullptr || cand == nullptr || picks == nullptr) return IQ_EINVAL;
+    if (rows <= 0 || nblk <= 0) return IQ_ESHAPE;
+    if (ldw < nblk * 256 || ldw % 8 != 0 || !aligned(w, 16) || !aligned(hess, 16)) return IQ_EINVAL;
+    if (cand_ld < nblk || cand_choice_stride < 0) return IQ_EINVAL;
+    if (!aligned(cand, 2) || (cand_choice_stride & 1) != 0) return IQ_EINVAL;  // 2-byte staging
+    if (rows_per_hess == 0) rows_per_hess = rows;
+    if (rows_per_hess < 0 || rows % rows_per_hess != 0) return IQ_ESHAPE;
+    int sms = 0;
+    if ((st = device_sms(&sms)) != IQ_OK) return st;
+    if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
+    iqk::ChoiceParams p;
+    p.w = w;
+    p.rows = rows;
+    p.nblk = nblk;
+    p.ldw = ldw;
+    p.hess = hess;
+    p.rows_per_hess = rows_per_hess;
+    p.cand = cand + iqk::kChoiceG8FirstLs * cand_choice_stride;  // the candidate for ls = 8
+    p.cand_ld = cand_ld;
+    p.cand_cstride = cand_choice_stride;
+    p.picks = picks;
+    p.payload = nullptr;
+    p.payload_ld = 0;
+    p.objective = objective;
+    p.flags = flags;
+    p.grid = desc->grid;
+    return launched(iqk::launch_choice_search(iqk::kChoiceIq2xsG8, p, sms, stream));
+}
+
 iq_status iq_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t stream) {
     if (hess == nullptr || out == nullptr) return IQ_EINVAL;
     if (nblk <= 0) return IQ_ESHAPE;

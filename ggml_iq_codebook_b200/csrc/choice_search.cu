@@ -14,6 +14,8 @@
 // updates grad_i by an fma chain over the group's k. NaN and +inf scores never win.
 //
 // Formats: IQ1_S (8 groups of 32 columns), IQ2_XS and IQ2_S (16 groups of 16 columns), 16 choices;
+// and a layout with eight candidates per 8-weight group (IQ2_XS candidates for ls = 8..15 over 32
+// groups of 8 columns; picks only, since no payload stores a scale per 8 weights);
 // IQ1_M (16 groups of 16 columns, 8 choices). With 8 choices two lanes share a candidate and each
 // forms half of the group's H_gg u columns and half of each score's products; a 16-wide pairwise
 // tree ends by adding its two 8-wide subtrees, so the halves join with one shuffle and one add.
@@ -146,7 +148,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 
 #ifndef IQ_CHOICE_COLUMN_MAX_W16
-#define IQ_CHOICE_COLUMN_MAX_W16 12  // 16-column choice groups (IQ2_XS, IQ2_S), 16 rows per CTA
+#define IQ_CHOICE_COLUMN_MAX_W16 12  // 16- and 8-column choice groups, 16 rows per CTA
 #endif
 #ifndef IQ_CHOICE_COLUMN_MAX_W32
 #define IQ_CHOICE_COLUMN_MAX_W32 0  // 32-column choice groups (IQ1_S): always tiles (measured)
@@ -154,17 +156,20 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 template <int FMT>
 struct Cfg {
+    static constexpr bool G8 = FMT == kChoiceIq2xsG8;          // eight candidates per 8-weight group
+    static constexpr int DF = G8 ? IQ_FMT_IQ2_XS : FMT;         // the candidates' payload format
+    static constexpr int PICK0 = G8 ? kChoiceG8FirstLs : 0;     // reported pick of candidate 0
     static constexpr int R = FMT == IQ_FMT_IQ1_S ? 8 : 16;      // rows per CTA (shared-memory budget)
     static constexpr int T = R * 16;                            // threads: a half-warp per row
     static constexpr int RG = R / 4;                            // 4-row groups of the gradient tiles
-    static constexpr int G = FMT == IQ_FMT_IQ1_S ? 8 : 16;     // choice groups per block
+    static constexpr int G = FMT == IQ_FMT_IQ1_S ? 8 : G8 ? 32 : 16;  // choice groups per block
     static constexpr int W = kBlock / G;                        // columns per choice group
-    static constexpr int B = FMT == IQ_FMT_IQ1_S   ? kIq1sBytes
-                             : FMT == IQ_FMT_IQ1_M ? kIq1mBytes
-                             : FMT == IQ_FMT_IQ2_S ? kIq2sBytes
-                                                   : kIq2xsBytes;
-    static constexpr int E = FMT == IQ_FMT_IQ2_XS ? kIq2xsEntries : FMT == IQ_FMT_IQ2_S ? kIq2sEntries : kIq1sEntries;
-    static constexpr int NC = FMT == IQ_FMT_IQ1_M ? kIq1mChoices : kChoices;  // candidates per row
+    static constexpr int B = DF == IQ_FMT_IQ1_S   ? kIq1sBytes
+                             : DF == IQ_FMT_IQ1_M ? kIq1mBytes
+                             : DF == IQ_FMT_IQ2_S ? kIq2sBytes
+                                                  : kIq2xsBytes;
+    static constexpr int E = DF == IQ_FMT_IQ2_XS ? kIq2xsEntries : DF == IQ_FMT_IQ2_S ? kIq2sEntries : kIq1sEntries;
+    static constexpr int NC = FMT == IQ_FMT_IQ1_M ? kIq1mChoices : G8 ? 8 : kChoices;  // candidates per row
     static constexpr int SPLIT = kChoices / NC;                 // lanes per candidate
     static constexpr int WO = W / SPLIT;                        // group columns per lane
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
@@ -176,7 +181,7 @@ struct Cfg {
     static constexpr int oUR = oUT + W * R * 4;                   // float [R][W]: the same, by row
     static constexpr int oSw = oCurT + kBlock * R * 4;            // int [R]: row switched this step
     // update by column up to this many switched rows, else by tiles (either is bit-exact)
-    static constexpr int COLUMN_MAX = W == 16 ? IQ_CHOICE_COLUMN_MAX_W16 : IQ_CHOICE_COLUMN_MAX_W32;
+    static constexpr int COLUMN_MAX = W == 32 ? IQ_CHOICE_COLUMN_MAX_W32 : IQ_CHOICE_COLUMN_MAX_W16;
     static constexpr int oGrid = oSw + R * 4;                     // uint16 [E] element codes
     static constexpr int oRows = oGrid + (E * 2 + 15) / 16 * 16;  // per-row records
     static constexpr int rX = 0;                                  // bf16 [256]
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
 
     // ---- stage the grid codes, the row's x (bf16) and its candidate payloads (lanes past the
     // format's NC candidates stage zeros and never win)
-    for (int q = tid; q < C::E; q += kThreads) sgrid[q] = grid_code<FMT>(__ldg(reinterpret_cast<const int2*>(p.grid) + q));
+    for (int q = tid; q < C::E; q += kThreads) sgrid[q] = grid_code<C::DF>(__ldg(reinterpret_cast<const int2*>(p.grid) + q));
     if (active) {
         const uint4* xs = reinterpret_cast<const uint4*>(p.w + row * p.ldw + blk * kBlock);
         bool nonfinite = false;
@@ -328,7 +333,9 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
 #pragma unroll
         for (int t = 0; t < W / 8; ++t) {
             float xh[8], xv[8];
-            decode8<FMT>(cand + ch * C::B, sgrid, g, (g * W + 8 * t) >> 3, xh);
+            // decode8 takes the format's own choice group: for 8-column groups, the 16-column
+            // group that holds the scale nibble
+            decode8<C::DF>(cand + ch * C::B, sgrid, C::G8 ? (g >> 1) : g, (g * W + 8 * t) >> 3, xh);
             unpack8_bf16(reinterpret_cast<const uint4*>(xb)[(g * W) / 8 + t], xv);
 #pragma unroll
             for (int j = 0; j < 8; ++j) dl[8 * t + j] = __fsub_rn(xv[j], xh[j]);
@@ -520,7 +527,9 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     // ---- step 4: picks and the payload assembled from the picked candidates
     if (active) {
         __syncwarp(hmask);
-        if (c < G) p.picks[(row * p.nblk + blk) * G + c] = static_cast<uint8_t>(pick[c]);
+        for (int q = c; q < G; q += 16) p.picks[(row * p.nblk + blk) * G + q] = static_cast<uint8_t>(C::PICK0 + pick[q]);
+    }
+    if (!C::G8 && active) {  // 8-column groups report picks only: no payload stores their scales
         uint8_t* out = p.payload + (row * p.payload_ld + blk) * C::B;
         for (int i = c; i < C::B; i += 16) {
             uint8_t v;
@@ -593,6 +602,7 @@ cudaError_t launch_choice_search(int fmt, const ChoiceParams& p, int /*num_sms*/
     if (fmt == IQ_FMT_IQ1_S) return launch<IQ_FMT_IQ1_S>(p, s);
     if (fmt == IQ_FMT_IQ2_S) return launch<IQ_FMT_IQ2_S>(p, s);
     if (fmt == IQ_FMT_IQ1_M) return launch<IQ_FMT_IQ1_M>(p, s);
+    if (fmt == kChoiceIq2xsG8) return launch<kChoiceIq2xsG8>(p, s);
     return launch<IQ_FMT_IQ2_XS>(p, s);
 }
 

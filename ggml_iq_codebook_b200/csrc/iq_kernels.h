@@ -46,6 +46,12 @@ struct ChoiceParams {
     const int8_t* grid;
 };
 
+// Choice-search layout code beside the iq_format values (not a payload format): IQ2_XS
+// candidates searched over 32 groups of 8 columns, eight candidates (ls = 8..15) per group,
+// picks only. The caller points cand at the candidate for ls = 8.
+constexpr int kChoiceIq2xsG8 = 5;
+constexpr int kChoiceG8FirstLs = 8;
+
 // Each returns the cudaError_t of its launch (cudaSuccess when nothing had to run).
 cudaError_t launch_iq1_encode(int fmt, const EncodeParams& p, int mode, int num_sms, cudaStream_t s);
 cudaError_t launch_iq2_encode(int fmt, const EncodeParams& p, int mode, int num_sms, cudaStream_t s);

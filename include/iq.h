@@ -193,6 +193,21 @@ iq_status iq_choice_search(const iq_desc *desc, const uint16_t *w, int64_t rows,
                            int64_t payload_ld, float *objective, uint32_t *flags, cudaStream_t stream);
 
 /*
+ * The same search with eight candidates per 8-weight group: 32 groups of 8 columns per block,
+ * each choosing among the IQ2_XS every-choice decodes for ls = 8..15 (PR #3158's steps, only the
+ * grouping differs; the 16-column search above is IQ2_XS's native one). desc must be IQ2_XS
+ * (IQ_EUNSUPPORTED otherwise). w, hess, rows_per_hess, objective and flags as above.
+ *   cand: the 16-choice IQ2_XS every-choice payloads, addressed as above; only choices 8..15 are
+ *     read.
+ *   picks: uint8 [rows][nblk][32], the chosen ls (8..15) of every 8-column group.
+ * No payload is written: no IQ layout stores a scale per 8 weights.
+ */
+iq_status iq_choice_search_g8(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t nblk, int64_t ldw,
+                              const float *hess, int64_t rows_per_hess, const uint8_t *cand, int64_t cand_ld,
+                              int64_t cand_choice_stride, uint8_t *picks, float *objective, uint32_t *flags,
+                              cudaStream_t stream);
+
+/*
  * out[b * 256 + i] = sqrtf(hess[b][i][i]) for b < nblk: the search importance the local-Hessian
  * calibration uses for the every-choice candidates (square root of the Hessian diagonal, PR #3158).
  */

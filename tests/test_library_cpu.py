@@ -23,7 +23,7 @@ def lib():
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "iq.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(iq_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(iq_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_binding_symbols():
@@ -99,5 +99,15 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert lib.iq_choice_search(ctypes.byref(m), W, 4, 1, 256, W, 3, W, 1, 0, W, W, 1, None, None, None) == 2  # 3 !| 4
     s2 = _desc(fmt=4, entries=1024, anchor=0.9)
     assert lib.iq_choice_search(ctypes.byref(s2), W, 0, 1, 256, W, 0, W, 1, 0, W, W, 1, None, None, None) == 2
+    # the 8-column choice search: IQ2_XS only; shapes and buffers as the 16-column one, no payload
+    x2 = _desc(fmt=2, entries=512, anchor=0.9)
+    G8 = lib.iq_choice_search_g8
+    assert G8(ctypes.byref(d), W, 4, 1, 256, W, 0, W, 1, 0, W, None, None, None) == 4
+    assert G8(ctypes.byref(x2), W, 0, 1, 256, W, 0, W, 1, 0, W, None, None, None) == 2
+    assert G8(ctypes.byref(x2), W, 6, 1, 256, W, 4, W, 1, 0, W, None, None, None) == 2  # 4 !| 6
+    assert G8(ctypes.byref(x2), W, 4, 1, 256, W, 0, W, 1, 0, None, None, None, None) == 1
+    assert G8(ctypes.byref(x2), W, 4, 2, 256, W, 0, W, 2, 0, W, None, None, None) == 1  # ldw < 512
+    assert G8(ctypes.byref(x2), W, 4, 1, 256, W, 0, W + 1, 1, 0, W, None, None, None) == 1
+    assert G8(ctypes.byref(x2), W, 4, 1, 256, W, 0, W, 1, 3, W, None, None, None) == 1
     assert lib.iq_sqrt_diag(None, 1, W, None) == 1
     assert lib.iq_sqrt_diag(W, 0, W, None) == 2
