@@ -244,6 +244,36 @@ def test_choice_search_matches_oracle(dev, descs, grids, anchors, fmt, offdiag):
     assert np.array_equal(pay.cpu().numpy(), want_pay)
 
 
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m", "g8"])
+def test_choice_search_exact_ties_match_oracle(dev, grids, anchors, fmt):
+    """Candidates duplicated at higher choices (exact ties in every score and gain), and all
+    candidates equal: picks, payload and objective bits as the oracle's (the lowest choice wins
+    ties, and a zero gain never switches). g8: eight candidates per 8-weight group."""
+    efmt = "iq2_xs" if fmt == "g8" else fmt
+    desc = iq.make_desc(efmt, torch.from_numpy(grids[efmt]).to(dev), anchors[efmt])
+    rows, nblk = 13, 2
+    w, hess = _choice_case(efmt, rows, nblk, 521, 0.3)
+    imp = oracle.sqrt_diag(hess.numpy())
+    cand, _ = oracle.encode(efmt, grids[efmt], anchors[efmt], w, importance=imp, every_choice=True)
+    C, lo = cand.shape[0], (8 if fmt == "g8" else 0)
+    dup = cand.copy()
+    dup[C - 1], dup[lo + 4] = dup[lo + 1], dup[lo + 2]
+    same = np.broadcast_to(cand[lo:lo + 1], cand.shape).copy()
+    for cd in (dup, same):
+        cdev = torch.from_numpy(cd).to(dev)
+        obj = torch.empty((rows, nblk), dtype=torch.float32, device=dev)
+        if fmt == "g8":
+            picks = iq.iq_choice_search_g8(desc, w.to(dev), hess.to(dev), cdev, objective=obj)
+            want_p, want_obj = oracle.choice_search_g8(grids["iq2_xs"], w, hess.numpy(), cd, objective=True)
+        else:
+            picks, pay = iq.iq_choice_search(desc, w.to(dev), hess.to(dev), cdev, objective=obj)
+            want_p, want_pay, want_obj = oracle.choice_search(fmt, grids[fmt], w, hess.numpy(), cd, objective=True)
+            assert np.array_equal(pay.cpu().numpy(), want_pay)
+        assert np.array_equal(picks.cpu().numpy(), want_p)
+        assert np.array_equal(obj.cpu().numpy().view(np.uint32), want_obj.view(np.uint32))
+        assert not (want_p == C - 1).any() and not (want_p == lo + 4).any()
+
+
 @pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s"])
 def test_local_hessian_pipeline_on_gpu_matches_oracle(dev, descs, grids, anchors, fmt):
     """sqrt(diag H) -> every-choice encode -> choice search, all in the library's kernels."""

@@ -614,3 +614,30 @@ def test_iq2xs_joint_enumeration_on_a_reduced_grid(anchors):
         got = sum(float(((xs[i] - s * grid[idx[2 * k + i]] * signs[2 * k + i]) ** 2 * ws[i]).sum()) for i in range(2))
         assert got <= best + 2e-5 * float((ws * xs ** 2).sum()), (k, got, best)
         assert idx[2 * k] < 16 and idx[2 * k + 1] < 16
+
+
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "iq2_s", "iq1_m", "g8"])
+def test_choice_search_ties_go_to_the_lowest_choice(grids, anchors, fmt):
+    """PR #3158's tie rules on exact ties: a candidate duplicated at a higher choice scores and
+    gains exactly what its lower copy does, so it is never picked (lowest choice on equal score,
+    and a switch needs a strictly negative gain); with every candidate equal nothing moves."""
+    efmt = "iq2_xs" if fmt == "g8" else fmt
+    w, hess, cand = _choice_case(efmt, grids, anchors, 4, 2, 161, 0.3)
+    C = cand.shape[0]
+    lo = 8 if fmt == "g8" else 0                      # first candidate the search reads
+
+    def search(cd):
+        if fmt == "g8":
+            return oracle.choice_search_g8(grids["iq2_xs"], w, hess, cd, trace=True)[1]
+        return oracle.choice_search(fmt, grids[fmt], w, hess, cd, trace=True)[2]
+
+    dup = cand.copy()
+    pairs = [(lo + 1, C - 1), (lo + 2, lo + 4)]       # (kept copy, higher duplicate)
+    for keep, high in pairs:
+        dup[high] = dup[keep]
+    tr = search(dup)
+    for _, high in pairs:
+        assert not (tr == high).any(), high
+    same = np.broadcast_to(cand[lo:lo + 1], cand.shape).copy()
+    tr = search(same)
+    assert (tr == lo).all()
