@@ -18,7 +18,9 @@
  *     1024-entry grid with eight sign bits for each group (the input's signs, no parity flip);
  *   - decoding of the four layouts;
  *   - the local-Hessian choice search (PR #3158, fused in PR #3218 "[4/4] Run the local-Hessian
- *     choice search as one CUDA kernel").
+ *     choice search as one CUDA kernel"), and the same search over eight candidates per 8-weight
+ *     group;
+ *   - encoding under given block scales (PR #3197, static scales).
  *
  * The exact floating-point op sequence of every score is a fixed convention (it is what makes
  * payloads and picks bit-reproducible); it is documented next to each kernel.
