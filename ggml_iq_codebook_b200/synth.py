@@ -10,7 +10,8 @@ Recipes (all seeded, all reproducible):
   rejected in draw order. The real GGML tables are third-party data and are not used.
 * IQ2_XS grid: 512 distinct 8-vectors over {1, 3, 5, 7}, drawn the same way.
 * Weights: i.i.d. normal in fp32, rounded to bf16 (round to nearest even). Outlier columns are
-  scaled by 8 after the rounding, which is exact in bf16.
+  scaled by 8 after the rounding, which is exact in bf16. A stack of expert weights draws expert e
+  from its own CPU generator (seed * 1024 + e), so any expert can be rebuilt on the host alone.
 * Importance: per input column, log-normal(0, 1) in fp64, stored as fp32; the square-root
   variant is the square root of a log-normal Hessian diagonal.
 * Block Hessian: H = U^-1 U^-T for an upper-triangular U with diagonal uniform in [0.5, 2] and
@@ -68,6 +69,20 @@ def normal_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
     g = torch.Generator(device=device).manual_seed(seed)
     x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
     return (x * std).to(torch.bfloat16)
+
+
+def normal_bf16_experts(experts: int, rows: int, cols: int, std: float, seed: int, device="cpu") -> torch.Tensor:
+    """[experts, rows, cols] bf16: expert e is normal_bf16((rows, cols), std, seed * 1024 + e) drawn
+    on the host, then moved to `device` one expert at a time."""
+    out = torch.empty((experts, rows, cols), dtype=torch.bfloat16, device=device)
+    for e in range(experts):
+        out[e].copy_(expert_bf16(e, rows, cols, std, seed))
+    return out
+
+
+def expert_bf16(e: int, rows: int, cols: int, std: float, seed: int) -> torch.Tensor:
+    """Expert e of normal_bf16_experts, on the host."""
+    return normal_bf16((rows, cols), std, seed * 1024 + e)
 
 
 def outlier_columns(cols: int, frac: float, seed: int) -> torch.Tensor:
@@ -140,10 +155,11 @@ def workload_iq2xs_8192x4096(device="cpu", rows=8192, cols=4096):
 
 
 def workload_iq1s_moe(device="cpu", experts=256, rows=1536, cols=4096):
-    """MoE batch: `experts` weights of rows x cols, N(0, 0.02^2), per-expert log-normal importance."""
+    """MoE batch: `experts` weights of rows x cols, N(0, 0.02^2), each expert drawn on the host from
+    its own seed (1004 * 1024 + e); per-expert log-normal importance."""
     return {
         "fmt": "iq1_s",
-        "w": normal_bf16((experts, rows, cols), 0.02, 1004, device),
+        "w": normal_bf16_experts(experts, rows, cols, 0.02, 1004, device),
         "importance": lognormal((experts, cols), 3004, device),
     }
 

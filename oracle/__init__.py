@@ -34,6 +34,7 @@ FLAG_NONFINITE = 1
 FLAG_IMPORTANCE = 2
 FLAG_RANGE = 4
 FLAG_CHOICE = 8
+FLAG_GRID = 16
 
 _lib = None
 
@@ -48,6 +49,19 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def build_optimised() -> str:
+    """The same source compiled with -O3 -march=native, still with -ffp-contract=off and without
+    fast-math, so IEEE semantics (and every output bit) are the plain build's. It serves only the
+    script that writes the stored full-size digests, where the plain build would take hours."""
+    out = os.path.join(_HERE, "liboracle_O3.so")
+    if not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-std=c11", "-O3", "-march=native", "-Wall", "-ffp-contract=off", "-fno-fast-math",
+               "-fopenmp", "-shared", "-fPIC", "-o", out + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(out + ".tmp", out)
+    return out
+
+
 def _load(path: str | None = None):
     global _lib
     if _lib is None or path is not None:
@@ -59,7 +73,7 @@ def _load(path: str | None = None):
                                    P, P]
         lib.orc_decode.restype = None
         lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
-        lib.orc_choice_search.restype = None
+        lib.orc_choice_search.restype = ctypes.c_uint32
         lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, i64, P, P, P, P, P]
         lib.orc_sqrt_diag.restype = None
         lib.orc_sqrt_diag.argtypes = [P, i64, P]
@@ -187,7 +201,7 @@ def decode(fmt: str, grid: np.ndarray, payload: np.ndarray) -> np.ndarray:
 
 
 def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False,
-                  objective=False):
+                  objective=False, return_flags=False):
     """Local-Hessian choice search over every 256-column block of w.
 
     w: [rows, cols], or [experts, rows, cols] with hess [experts, nblk, 256, 256] (each expert's
@@ -195,7 +209,10 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     cand: [C, (experts,) rows, nblk, B] every-choice payloads (C = 16; 8 for iq1_m).
     Returns (picks [(experts,) rows, nblk, G], payload [(experts,) rows, nblk, B]) and, with
     trace, the picks after step 2 and after each sweep [(experts,) rows, nblk, 3, G]; with objective
-    (last), each row-block's final Delta^T H Delta [(experts,) rows, nblk] fp32.
+    (after the picks and payload, or the trace), each row-block's final Delta^T H Delta
+    [(experts,) rows, nblk] fp32; with return_flags (last), the findings word (FLAG_NONFINITE for a
+    non-finite weight or Hessian entry, FLAG_GRID for a grid value outside the alphabet). A
+    row-block with a finding gets picks 0, the all-zero payload and a NaN objective.
     Parity of the sweeps is pinned by the fp64 direct-objective replay in the tests.
     """
     wb = _bf16_bits(w)
@@ -212,19 +229,21 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     payload = np.zeros((rows, nblk, B), dtype=np.uint8)
     tr = np.zeros((rows, nblk, 3, G), dtype=np.uint8) if trace else None
     obj = np.zeros((rows, nblk), dtype=np.float32) if objective else None
-    _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
-                              rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
-                              _ptr(payload), _ptr(tr), _ptr(obj))
+    flags = _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
+                                      rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
+                                      _ptr(payload), _ptr(tr), _ptr(obj))
     out = [picks.reshape(lead + (nblk, G)), payload.reshape(lead + (nblk, B))]
     if trace:
         out.append(tr.reshape(lead + (nblk, 3, G)))
     if objective:
         out.append(obj.reshape(lead + (nblk,)))
+    if return_flags:
+        out.append(int(flags))
     return tuple(out)
 
 
 def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, trace=False,
-                     objective=False):
+                     objective=False, return_flags=False):
     """The local-Hessian choice search with eight candidates per 8-weight group: 32 groups of 8
     columns per block, each choosing among the IQ2_XS every-choice decodes for ls = 8..15.
 
@@ -232,8 +251,9 @@ def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, tr
     [16, (experts,) rows, nblk, 74], of which choices 8..15 are read. Returns (picks,) with picks
     [(experts,) rows, nblk, 32] holding the chosen ls (8..15); with trace, also the picks after
     step 2 and after each sweep [(experts,) rows, nblk, 3, 32]; with objective (last), each
-    row-block's final Delta^T H Delta. No payload layout stores a scale per 8 weights, so none
-    is assembled.
+    row-block's final Delta^T H Delta; with return_flags (last), the findings word, as in
+    choice_search (a row-block with a finding gets picks 8). No payload layout stores a scale per
+    8 weights, so none is assembled.
     """
     wb = _bf16_bits(w)
     lead = wb.shape[:-1]
@@ -247,14 +267,16 @@ def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, tr
     picks = np.zeros((rows, nblk, 32), dtype=np.uint8)
     tr = np.zeros((rows, nblk, 3, 32), dtype=np.uint8) if trace else None
     obj = np.zeros((rows, nblk), dtype=np.float32) if objective else None
-    _load().orc_choice_search(CS_IQ2XS_G8, _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
-                              rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
-                              None, _ptr(tr), _ptr(obj))
+    flags = _load().orc_choice_search(CS_IQ2XS_G8, _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
+                                      rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
+                                      None, _ptr(tr), _ptr(obj))
     out = [picks.reshape(lead + (nblk, 32))]
     if trace:
         out.append(tr.reshape(lead + (nblk, 3, 32)))
     if objective:
         out.append(obj.reshape(lead + (nblk,)))
+    if return_flags:
+        out.append(int(flags))
     return tuple(out)
 
 
