@@ -39,24 +39,27 @@ METRIC = "IQ encode Mweights/s"
 UNIT = "Mweights/s"
 L2_FLUSH_BYTES = 256 << 20
 
-# FP32-pipe operations the method itself requires (the exhaustive search counts every candidate):
-#   IQ1_S, per (group, grid entry): 4 subset-sum adds + A, R, C (3) + A_delta, C_delta for both
-#     shifts (6 fma) = 13 term ops, then 16 choices x (1 fma score + 1 min) = 32 -> 45 ops;
-#     per 256-weight block: 32 groups x 2048 entries x 45 = 2,949,120 ops.
-#   IQ2_XS, per (group, entry): A and B chains (16) + 16 x (fma + min) = 48 ops;
-#     per block: 32 x 512 x 48 = 786,432 ops.
-#   Choice search (G choice groups of W = 256 / G columns, C choices), per row and block:
-#     own-block scores G x C x (W^2 + 2W - 1), gradient 256 x 256, two sweeps of
-#     G x C x (W^2 + 5W - 1) gains; gradient updates after a switch are data dependent and not
-#     counted. IQ2_XS and IQ2_S (G = C = 16): 310,528 ops; IQ1_S (G = 8, C = 16): 507,520 ops;
-#     IQ1_M (G = 16, C = 8): 188,032 ops; eight candidates per 8-weight group (G = 32, C = 8):
-#     138,496 ops.
-#   IQ1_M runs IQ1_S's search (same 2048 x 16 candidates per group): 2,949,120 ops per block.
-#   IQ2_S runs IQ2_XS's per-entry work over 1024 entries: 32 x 1024 x 48 = 1,572,864 per block.
-OPS_PER_BLOCK = {"iq1_s": 2_949_120, "iq2_xs": 786_432, "iq1_m": 2_949_120, "iq2_s": 1_572_864}
+# FP32 operations the method itself requires, counted as the survey's work table counts them
+# (every candidate of the exhaustive search counts, an fma and a min one op each):
+#   IQ1_S, per 8-weight group: 2048 entries x 16 choices = 32,768 candidates x (fma + min) plus
+#     about 10 entry-term ops per entry (2048 x 10) = 86,016 ops; per 256-weight block x32 =
+#     2,752,512. IQ1_M runs the same search.
+#   IQ2_XS, per group: 8,192 candidates x (fma + min) + 512 x 16 fma for A and B = 24,576 ops;
+#     per block 786,432. IQ2_S runs it over 1024 entries: 1,572,864 per block.
+#   Choice search (G groups of W = 256 / G columns, C choices), per row and block: H Delta
+#     (256 x 256 fma) + the own-block scores G x C x (W^2 + W) + two sweeps, each group step
+#     counted as C x (W^2 + W) gain products plus a full 256 x W gradient update:
+#     65,536 + G C (W^2 + W) + 2 G (C (W^2 + W) + 256 W). IQ2_XS and IQ2_S: 405,504;
+#     IQ1_S (8, 32, 16): 602,112; IQ1_M (16, 16, 8): 301,056; eight candidates per 8-weight group
+#     (32, 8, 8): 251,904.
+OPS_PER_BLOCK = {"iq1_s": 2_752_512, "iq2_xs": 786_432, "iq1_m": 2_752_512, "iq2_s": 1_572_864}
+
+
 def choice_ops_per_row_block(G: int, C: int = 16) -> int:
     W = 256 // G
-    return G * C * (W * W + 2 * W - 1) + 256 * 256 + 2 * G * C * (W * W + 5 * W - 1)
+    return 256 * 256 + G * C * (W * W + W) + 2 * G * (C * (W * W + W) + 256 * W)
+
+
 SMS, FP32_LANES = 148, 128
 
 
@@ -70,6 +73,39 @@ def load_peaks():
 
 def alu_peak_tops(mhz: float) -> float:
     return SMS * FP32_LANES * mhz * 1e6 / 1e12
+
+
+def measure_fp32(dev, kinds=("ffma", "ffma2", "candidate_mix", "candidate_mix_ffma2"), reps=5, iters=200_000):
+    """FP32 lane ops/s (T/s) of each probe kind: 8 CTAs of 256 threads per SM, CUDA events on the
+    launching stream, median of `reps` launches after one warm-up."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks = 8 * sms
+    out = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    rates = {}
+    for kind in kinds:
+        iq.probe_fp32(kind, blocks, iters // 10, out)
+        times = []
+        for _ in range(reps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            ops = iq.probe_fp32(kind, blocks, iters, out)
+            e.record()
+            torch.cuda.synchronize()
+            times.append(s.elapsed_time(e))
+        rates[kind] = round(ops / (statistics.median(times) / 1e3) / 1e12, 3)
+    return rates
+
+
+def fp32_peak_line(args, dev):
+    """--workload fp32_peak: the probe rates as one JSON line, with the clocks seen."""
+    with Clocks(torch.cuda.current_device()) as clk:
+        rates = measure_fp32(dev)
+    clocks = clk.summary()
+    nominal = alu_peak_tops(clocks["sm_max_mhz"] if clocks and clocks["sm_max_mhz"] else 1965.0)
+    print(json.dumps({"metric": "FP32 lane ops/s", "unit": "Top/s", "rates": rates,
+                      "peak": max(rates["ffma"], rates["ffma2"]), "nominal_lanes_x_clock": round(nominal, 3),
+                      "clocks": clocks, "probe": "iq_probe_fp32, 8 CTAs x 256 threads per SM, 8 chains/thread"}),
+          flush=True)
 
 
 def kernel_traffic(name: str, workload: str, blocks: int):
@@ -209,6 +245,9 @@ class Workload:
         self.desc = {"iq1_s": iq.make_desc("iq1_s", g1), "iq2_xs": iq.make_desc("iq2_xs", g2),
                      "iq1_m": iq.make_desc("iq1_m", g1), "iq2_s": iq.make_desc("iq2_s", g3)}
         self.launches_per_step = 2
+        # the kernels' findings word: kept on the device during the timed steps (no host round
+        # trip per call) and checked once afterwards
+        self.flags = torch.zeros(1, dtype=torch.int32, device=dev)
         if name not in WORKLOADS:
             raise SystemExit(f"unknown workload {name}")
         text = WORKLOADS[name][2]
@@ -294,24 +333,26 @@ class Workload:
         elif self.kind == "encode":
             if ev is not None:
                 ev[0].record()
-            iq.iq_encode(d, self.w, self.imp, out=self.payload, flags=False)
+            iq.iq_encode(d, self.w, self.imp, out=self.payload, flags=self.flags, raise_on_flags=False)
             if ev is not None:
                 ev[1].record()
             iq.iq_decode(d, self.payload, torch.bfloat16, out=self.decoded)
         else:
             iq.iq_sqrt_diag(self.hess, out=self.imp)
-            iq.iq_encode(d, self.w, self.imp, every_choice=True, out=self.cand, flags=False)
+            iq.iq_encode(d, self.w, self.imp, every_choice=True, out=self.cand, flags=self.flags,
+                         raise_on_flags=False)
             if ev is not None:
                 ev[0].record()
             if self.per_block:  # one call per 256-column block, on views into the whole-weight tensors
                 for b in range(self.w.shape[-1] // 256):
                     iq.iq_choice_search(d, self.w[:, 256 * b:256 * (b + 1)], self.hess[b:b + 1],
                                         self.cand[:, :, b:b + 1], picks=self.picks_b[b],
-                                        payload=self.payload[:, b:b + 1])
+                                        payload=self.payload[:, b:b + 1], flags=self.flags)
             elif self.g8:
-                iq.iq_choice_search_g8(d, self.w, self.hess, self.cand, picks=self.picks)
+                iq.iq_choice_search_g8(d, self.w, self.hess, self.cand, picks=self.picks, flags=self.flags)
             else:
-                iq.iq_choice_search(d, self.w, self.hess, self.cand, picks=self.picks, payload=self.payload)
+                iq.iq_choice_search(d, self.w, self.hess, self.cand, picks=self.picks, payload=self.payload,
+                                    flags=self.flags)
             if ev is not None:
                 ev[1].record()
 
@@ -326,7 +367,7 @@ class Workload:
             self.w.copy_(host["w"], non_blocking=True)
             if self.imp is not None:
                 self.imp.copy_(host["imp"], non_blocking=True)
-            iq.iq_encode(d, self.w, self.imp, out=self.payload, flags=False)
+            iq.iq_encode(d, self.w, self.imp, out=self.payload, flags=self.flags, raise_on_flags=False)
             iq.iq_decode(d, self.payload, torch.bfloat16, out=self.decoded)
             host["payload"].copy_(self.payload, non_blocking=True)
             host["decoded"].copy_(self.decoded, non_blocking=True)
@@ -423,7 +464,7 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
         cols = w.shape[1]
     else:
         if name == "iq1s_moe_256x1536x4096":
-            w, imp = synth.normal_bf16((1536, 4096), 0.02, 1004), synth.lognormal((256, 4096), 3004)[0]
+            w, imp = synth.expert_bf16(0, 1536, 4096, 0.02, 1004), synth.lognormal((256, 4096), 3004)[0]
             fmt = "iq1_s"
         else:
             wl = {"iq1s_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
@@ -486,7 +527,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
-    ap.add_argument("--workload", default="iq1s_4096x4096_weighted")
+    ap.add_argument("--workload", default="iq1s_moe_256x1536x4096")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -496,6 +537,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     peaks = load_peaks()
+    if args.workload == "fp32_peak":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        iq.load_library()
+        if rank == 0:
+            fp32_peak_line(args, dev)
+        return
     if args.workload not in WORKLOADS:
         raise SystemExit(f"unknown workload {args.workload}")
     fmt, shape, text = WORKLOADS[args.workload]
@@ -541,6 +589,7 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    iq.raise_for_flags(wl.flags)  # the timed steps' findings (none on these inputs)
     step_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in step_ev), dist, dev)
     dom_ms = [s.elapsed_time(e) for s, e in dom_ev]
     ms_per_step = step_ms / args.steps
@@ -562,6 +611,7 @@ def main():
     e2e_value = weak_scaling_value(wl.units, world, e2e_ms)
 
     dec = decode_roofline(wl, dev, peaks) if rank == 0 else None
+    fp32 = measure_fp32(dev, kinds=("ffma", "ffma2"), reps=3) if rank == 0 and wl.kind != "decode" else None
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -579,13 +629,18 @@ def main():
                 "traffic_source": tnote, "bytes_per_launch": nbytes, "ms_per_launch": round(dom_avg, 4)}
     else:
         achieved = wl.ops_per_launch / (dom_avg / 1e3) / 1e12
-        peak = alu_peak_tops(peaks["sm_max_mhz"])
-        roof = {"bound": "alu", "kernel": wl.dominant, "achieved": round(achieved, 3), "peak": round(peak, 3),
+        peak = max(fp32.values())
+        nominal = alu_peak_tops(peaks["sm_max_mhz"])
+        roof = {"bound": "alu", "kernel": wl.dominant, "achieved": round(achieved, 3), "peak": peak,
                 "unit": "Top/s", "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_source": tnote,
-                "ops_per_launch": wl.ops_per_launch, "ms_per_launch": round(dom_avg, 4),
-                "peak_basis": f"{SMS} SMs x {FP32_LANES} FP32 lanes x {peaks['sm_max_mhz']:.0f} MHz (1 op/lane/clock)"}
-        if clocks:
-            roof["frac_at_measured_clock"] = round(achieved / alu_peak_tops(clocks["sm_mhz"]), 4)
+                "ops_per_launch": wl.ops_per_launch, "ops_count": "the survey's work table (every candidate "
+                "counts; fma and min one op each)", "ms_per_launch": round(dom_avg, 4),
+                "peak_basis": "measured in this run: FP32 lane ops/s of iq_probe_fp32 (8 CTAs x 256 threads per "
+                f"SM), the larger of scalar fma {fp32['ffma']} and packed fma.f32x2 {fp32['ffma2']} Top/s",
+                "peak_nominal": round(nominal, 3), "frac_of_nominal": round(achieved / nominal, 4)}
+        if wl.kind == "choice":
+            roof["ops_executed_note"] = ("the count includes a gradient update after every group step; the "
+                                         "kernel updates only after a switch")
 
     cpu = None
     if not args.no_cpu_baseline:

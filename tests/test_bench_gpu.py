@@ -40,7 +40,15 @@ def test_bench_line(workload):
         assert line["decode"]["achieved_gbs"] > 0
 
 
+def test_bench_fp32_peak_probe():
+    line = _run("--workload", "fp32_peak")
+    rates = line["rates"]
+    assert set(rates) == {"ffma", "ffma2", "candidate_mix", "candidate_mix_ffma2"}
+    assert all(v > 0 for v in rates.values()) and line["peak"] == max(rates["ffma"], rates["ffma2"])
+
+
 def test_bench_default_with_cpu_baseline():
     line = _run("--steps", "3", "--warmup", "3")
-    assert line["config"]["workload"] == "iq1s_4096x4096_weighted"
+    assert line["config"]["workload"] == "iq1s_moe_256x1536x4096"
+    assert "measured in this run" in line["roofline"]["peak_basis"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
