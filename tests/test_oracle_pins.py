@@ -211,27 +211,52 @@ def test_iq2xs_search_reaches_bruteforce_minimum(grids, anchors, weighted):
 # ------------------------------------------------------------------------------ invariants
 
 def test_iq1s_fields_not_degenerate(grids, anchors):
-    """PR #2450 review: indices address the grid, ls and delta take several values, d > 0."""
+    """PR #2450 review: ls and delta take several values, d > 0, and the index fields are really
+    used: their high bits (qh bits 0..11) take several values, and every group's decoded entry
+    has the sign pattern the group's weights ask for more often than chance (an index read from
+    the wrong bits addresses an unrelated grid row)."""
     wl = synth.workload_iq1s_64x256()
     p, flags = oracle.encode("iq1_s", grids["iq1_s"], anchors["iq1_s"], wl["w"])
     assert flags == 0
+    x = wl["w"].float().numpy().reshape(-1, 256)
     f = [iq1s_fields(b) for b in p.reshape(-1, 50)]
     assert all(fi[0] > 0 for fi in f)
-    assert max(fi[3].max() for fi in f) < 2048
+    assert len(np.unique(np.concatenate([fi[3] >> 8 for fi in f]))) > 4
     assert len(np.unique(np.concatenate([fi[1] for fi in f]))) > 1
     assert len(np.unique(np.concatenate([fi[2] for fi in f]))) == 2
+    # the entry of a group tracks the signs of its largest weights: count, over all groups, the
+    # elements whose grid value has the weight's sign among the 2 largest |x| of the group
+    agree = total = 0
+    for blk, fi in zip(x, f):
+        q = grids["iq1_s"][fi[3]].astype(np.int64)  # [32, 8]
+        xg = blk.reshape(32, 8)
+        top = np.argsort(-np.abs(xg), axis=1)[:, :2]
+        for g in range(32):
+            for j in top[g]:
+                total += 1
+                agree += int(np.sign(q[g, j]) == np.sign(xg[g, j]))
+    assert agree > 0.8 * total, (agree, total)
 
 
 def test_iq2xs_fields_not_degenerate(grids, anchors):
-    """PR #2450 review: parity holds (signs match x up to one flip), nibbles not all equal, d > 0."""
+    """PR #2450 review: the decoded signs are the input's signs up to the one weakest flip an odd
+    count needs, the scale nibbles are not all equal, the 9-bit indices use their top bit, and
+    d > 0."""
     w, imp = _case(16, 256, 51, std=0.015)
     p, flags = oracle.encode("iq2_xs", grids["iq2_xs"], anchors["iq2_xs"], w, importance=imp)
     assert flags == 0
-    for blk in p.reshape(-1, 74):
+    x = w.float().numpy().reshape(-1, 256)
+    tops = set()
+    for blk, xb in zip(p.reshape(-1, 74), x):
         d, ls, idx, s7 = iq2xs_fields(blk)
         assert d > 0
         assert len(np.unique(ls)) > 1
-        assert (iq2xs_signs(s7) < 0).sum(-1).max() <= 8
+        tops |= set((idx >> 8).tolist())
+        dec_neg = iq2xs_signs(s7) < 0           # [32, 8]
+        in_neg = xb.reshape(32, 8) < 0
+        diff = (dec_neg != in_neg).sum(-1)      # elements whose sign the encoder changed
+        assert np.array_equal(diff, in_neg.sum(-1) % 2), (diff, in_neg.sum(-1))
+    assert tops == {0, 1}
 
 
 @pytest.mark.parametrize("fmt", ["iq1_s", "iq2_xs"])
@@ -641,3 +666,44 @@ def test_choice_search_ties_go_to_the_lowest_choice(grids, anchors, fmt):
     same = np.broadcast_to(cand[lo:lo + 1], cand.shape).copy()
     tr = search(same)
     assert (tr == lo).all()
+
+
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s", "g8"])
+def test_choice_search_findings_policy(grids, anchors, fmt):
+    """A non-finite weight taints its own row-block, a non-finite Hessian entry every row-block of
+    that Hessian block, a grid value outside the alphabet every block: those get picks 0 (the first
+    candidate), the all-zero payload and a NaN objective, with the finding flagged; the other
+    row-blocks are exactly what they are without the bad input."""
+    base = "iq2_xs" if fmt == "g8" else fmt
+    w, hess, cand = _choice_case(base, grids, anchors, 4, 2, 131, 0.3)
+
+    def run(w_, h_, g_):
+        if fmt == "g8":
+            picks, obj, flags = oracle.choice_search_g8(g_, w_, h_, cand, objective=True, return_flags=True)
+            return picks, None, obj, flags
+        return oracle.choice_search(fmt, g_, w_, h_, cand, objective=True, return_flags=True)
+
+    picks0, pay0, obj0, f0 = run(w, hess, grids[base])
+    assert f0 == 0
+    first = 8 if fmt == "g8" else 0
+    nan_bits = np.uint32(0x7FC00000)
+    wb = w.clone()
+    wb[1, 300] = float("nan")                      # row 1, block 1
+    hb = hess.copy()
+    hb[0, 7, 9] = np.inf                           # block 0 of every row
+    picks, pay, obj, f = run(wb, hb, grids[base])
+    assert f == oracle.FLAG_NONFINITE
+    bad = np.zeros((4, 2), bool)
+    bad[:, 0] = True
+    bad[1, 1] = True
+    assert np.all(picks[bad] == first) and np.all(obj.view(np.uint32)[bad] == nan_bits)
+    assert np.array_equal(picks[~bad], picks0[~bad]) and np.array_equal(obj[~bad], obj0[~bad])
+    if pay is not None:
+        assert not pay[bad].any() and np.array_equal(pay[~bad], pay0[~bad])
+    g_bad = grids[base].copy()
+    g_bad[3, 2] = 2 if base != "iq1_s" else -2     # outside {1,3,5,7} / {-1,0,1}
+    picks, pay, obj, f = run(w, hess, g_bad)
+    assert f == oracle.FLAG_GRID
+    assert np.all(picks == first) and np.all(obj.view(np.uint32) == nan_bits)
+    if pay is not None:
+        assert not pay.any()
