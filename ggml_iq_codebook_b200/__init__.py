@@ -33,8 +33,9 @@ IQ_OUT_F32, IQ_OUT_BF16 = 0, 1
 IQ_IN = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
 
-SYMBOLS = ("iq_block_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
+SYMBOLS = ("iq_block_bytes", "iq_payload_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
            "iq_choice_search", "iq_choice_search_g8", "iq_sqrt_diag", "iq_status_string", "iq_build_info")
+PROBE_SYMBOLS = ("iq_probe_fp32", "iq_probe_fp32_ops_per_iter")  # include/iq_probe.h: measurement only
 
 
 class IQError(RuntimeError):
@@ -60,6 +61,8 @@ def load_library(path: str = LIB_PATH):
     P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
     lib.iq_block_bytes.restype = ctypes.c_size_t
     lib.iq_block_bytes.argtypes = [i32]
+    lib.iq_payload_bytes.restype = ctypes.c_size_t
+    lib.iq_payload_bytes.argtypes = [i32, i64, i64]
     lib.iq_choice_groups.restype = i32
     lib.iq_choice_groups.argtypes = [i32]
     lib.iq_num_choices.restype = i32
@@ -79,6 +82,10 @@ def load_library(path: str = LIB_PATH):
     lib.iq_status_string.restype = ctypes.c_char_p
     lib.iq_status_string.argtypes = [ctypes.c_int]
     lib.iq_build_info.restype = ctypes.c_char_p
+    lib.iq_probe_fp32.restype = i32
+    lib.iq_probe_fp32.argtypes = [i32, i64, i64, P, P]
+    lib.iq_probe_fp32_ops_per_iter.restype = i64
+    lib.iq_probe_fp32_ops_per_iter.argtypes = [i32]
     _lib = lib
     return lib
 
@@ -126,8 +133,9 @@ def iq_encode(desc: IQDesc, w: torch.Tensor, importance: torch.Tensor | None = N
     IQ1_M, an existing payload uint8 [..., rows, cols/256, B] whose d fields are read in place.
     Returns the payload uint8 [(C,) (batch,) rows, cols/256, B], C = CHOICES[fmt]. With
     raise_on_flags (default) the call synchronises and raises on a device-side finding; pass a flags tensor and
-    raise_on_flags=False to stay asynchronous, or flags=False to skip the findings word
-    (invalid blocks are still written as zero payloads).
+    raise_on_flags=False to stay asynchronous. flags=False passes no findings word: the library
+    then synchronises itself and the call raises IQError with the finding's status (invalid
+    blocks are written as zero payloads either way).
     """
     lib = load_library()
     fmt = _fmt_of(desc)
@@ -241,6 +249,8 @@ def _choice_args(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand: torch.
     if w.dim() not in (2, 3) or w.stride(-1) != 1:
         raise IQError("w must be [rows, cols] or [experts, rows, cols] with a contiguous last dim")
     lead, cols = tuple(w.shape[:-1]), w.shape[-1]
+    if cols == 0 or cols % 256:
+        raise IQError(f"w must have a positive multiple of 256 columns, got {cols}")
     nexp, rows_e = (lead[0], lead[1]) if w.dim() == 3 else (1, lead[0])
     if w.dim() == 3 and nexp > 1 and w.stride(0) != rows_e * w.stride(1):
         raise IQError("the experts of w must be evenly spaced in the row dimension")
@@ -330,6 +340,21 @@ def iq_sqrt_diag(hess: torch.Tensor, out: torch.Tensor | None = None, stream=Non
         out = torch.empty(nblk * 256, dtype=torch.float32, device=hess.device)
     _check(lib.iq_sqrt_diag(hess.data_ptr(), nblk, out.data_ptr(), _stream(stream)))
     return out
+
+
+PROBE_KINDS = {"ffma": 0, "ffma2": 1, "candidate_mix": 2, "candidate_mix_ffma2": 3}
+
+
+def probe_fp32(kind: str, blocks: int, iters: int, out: torch.Tensor, stream=None) -> int:
+    """Launch the FP32 issue-rate probe (include/iq_probe.h); returns the lane ops it performs."""
+    lib = load_library()
+    _need(out, torch.float32, "out")
+    if out.numel() < blocks * 256:
+        raise IQError("out must hold blocks * 256 floats")
+    k = PROBE_KINDS[kind]
+    if lib.iq_probe_fp32(k, blocks, iters, out.data_ptr(), _stream(stream)) != 0:
+        raise IQError("iq_probe_fp32 failed")
+    return blocks * 256 * iters * int(lib.iq_probe_fp32_ops_per_iter(k))
 
 
 def build_info() -> str:

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI (include/iq.h): argument validation on the host, then kernel launches.
 #include <atomic>
 #include <cmath>
+#include <mutex>
 
 #include "iq.h"
 #include "iq_kernels.h"
@@ -56,6 +57,63 @@ iq_status launched(cudaError_t e) { return e == cudaSuccess ? IQ_OK : IQ_ECUDA; 
 
 }  // namespace
 
+// The findings word of calls made without one: one per device (a __device__ variable has an
+// instance on every device that loads the library). Such calls hold the device's mutex from
+// clearing the word to reading it back, so two of them never share it.
+__device__ uint32_t g_own_flags;
+
+namespace {
+
+std::mutex g_own_flags_mutex[kMaxDevices];
+
+// The flags word a call reports through: the caller's device word (cleared on the stream, read
+// by the caller), or, when the caller passes none, the library's own word, read back after the
+// stream has finished the call and turned into a status.
+class FlagsWord {
+  public:
+    explicit FlagsWord(uint32_t* caller) : caller_(caller) {}
+    ~FlagsWord() {
+        if (locked_) g_own_flags_mutex[dev_].unlock();
+    }
+    iq_status begin(cudaStream_t s) {
+        uint32_t* w = caller_;
+        if (w == nullptr) {
+            if (cudaGetDevice(&dev_) != cudaSuccess) return IQ_ECUDA;
+            if (dev_ < 0 || dev_ >= kMaxDevices) return IQ_EUNSUPPORTED;
+            g_own_flags_mutex[dev_].lock();
+            locked_ = true;
+            if (cudaGetSymbolAddress(reinterpret_cast<void**>(&own_), g_own_flags) != cudaSuccess) return IQ_ECUDA;
+            w = own_;
+        }
+        return cudaMemsetAsync(w, 0, sizeof(uint32_t), s) == cudaSuccess ? IQ_OK : IQ_ECUDA;
+    }
+    uint32_t* ptr() const { return caller_ != nullptr ? caller_ : own_; }
+    // The call's status: `st` itself when the launch failed or the caller keeps the word;
+    // otherwise the library's word is read once the stream is done, and a finding becomes
+    // IQ_EGRID, IQ_ENONFINITE, IQ_EIMPORTANCE, IQ_ERANGE or IQ_ECHOICE (first match wins).
+    iq_status finish(iq_status st, cudaStream_t s) {
+        if (st != IQ_OK || caller_ != nullptr) return st;
+        uint32_t f = 0;
+        if (cudaMemcpyAsync(&f, own_, sizeof(f), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return IQ_ECUDA;
+        if (f & IQ_FLAG_GRID) return IQ_EGRID;
+        if (f & IQ_FLAG_NONFINITE) return IQ_ENONFINITE;
+        if (f & IQ_FLAG_IMPORTANCE) return IQ_EIMPORTANCE;
+        if (f & IQ_FLAG_RANGE) return IQ_ERANGE;
+        if (f & IQ_FLAG_CHOICE) return IQ_ECHOICE;
+        return IQ_OK;
+    }
+
+  private:
+    uint32_t* caller_;
+    uint32_t* own_ = nullptr;
+    int dev_ = 0;
+    bool locked_ = false;
+};
+
+}  // namespace
+
 extern "C" {
 
 size_t iq_block_bytes(int32_t fmt) {
@@ -68,6 +126,12 @@ int32_t iq_choice_groups(int32_t fmt) {
 
 int32_t iq_num_choices(int32_t fmt) {
     return (fmt == IQ_FMT_IQ1_S || fmt == IQ_FMT_IQ2_XS || fmt == IQ_FMT_IQ2_S) ? 16 : fmt == IQ_FMT_IQ1_M ? 8 : 0;
+}
+
+size_t iq_payload_bytes(int32_t fmt, int64_t rows, int64_t cols) {
+    const size_t b = iq_block_bytes(fmt);
+    if (b == 0 || rows < 0 || cols < 0 || cols % 256 != 0) return 0;
+    return static_cast<size_t>(rows) * static_cast<size_t>(cols / 256) * b;
 }
 
 iq_status iq_encode(const iq_desc* desc, const void* w, int32_t w_dtype, int64_t batch, int64_t rows, int64_t cols,
@@ -92,7 +156,8 @@ iq_status iq_encode(const iq_desc* desc, const void* w, int32_t w_dtype, int64_t
         return IQ_EINVAL;
     int sms = 0;
     if ((st = device_sms(&sms)) != IQ_OK) return st;
-    if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
+    FlagsWord fw(flags);
+    if ((st = fw.begin(stream)) != IQ_OK) return st;
 
     iqk::EncodeParams p;
     p.w = w;
@@ -107,14 +172,15 @@ iq_status iq_encode(const iq_desc* desc, const void* w, int32_t w_dtype, int64_t
     p.scales = scales;
     p.scales_stride = scales != nullptr ? scales_stride : 0;
     p.payload = payload;
-    p.flags = flags;
+    p.flags = fw.ptr();
     p.grid = desc->grid;
     p.anchor = desc->anchor;
     p.nb = batch * rows * (cols / 256);
     const int mode = every_choice ? iqk::kEvery : (choices != nullptr ? iqk::kFixed : iqk::kSearch);
     const bool iq2 = desc->fmt == IQ_FMT_IQ2_XS || desc->fmt == IQ_FMT_IQ2_S;
-    return launched(iq2 ? iqk::launch_iq2_encode(desc->fmt, p, mode, sms, stream)
-                        : iqk::launch_iq1_encode(desc->fmt, p, mode, sms, stream));
+    return fw.finish(launched(iq2 ? iqk::launch_iq2_encode(desc->fmt, p, mode, sms, stream)
+                                  : iqk::launch_iq1_encode(desc->fmt, p, mode, sms, stream)),
+                     stream);
 }
 
 iq_status iq_decode(const iq_desc* desc, const uint8_t* payload, int64_t nblocks, int32_t out_dtype,
@@ -151,7 +217,8 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     if (rows_per_hess < 0 || rows % rows_per_hess != 0) return IQ_ESHAPE;
     int sms = 0;
     if ((st = device_sms(&sms)) != IQ_OK) return st;
-    if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
+    FlagsWord fw(flags);
+    if ((st = fw.begin(stream)) != IQ_OK) return st;
     iqk::ChoiceParams p;
     p.w = w;
     p.rows = rows;
@@ -166,9 +233,9 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     p.payload = payload;
     p.payload_ld = payload_ld;
     p.objective = objective;
-    p.flags = flags;
+    p.flags = fw.ptr();
     p.grid = desc->grid;
-    return launched(iqk::launch_choice_search(desc->fmt, p, sms, stream));
+    return fw.finish(launched(iqk::launch_choice_search(desc->fmt, p, sms, stream)), stream);
 }
 
 iq_status iq_choice_search_g8(const iq_desc* desc, const uint16_t* w, int64_t rows, int64_t nblk, int64_t ldw,
@@ -187,7 +254,8 @@ iq_status iq_choice_search_g8(const iq_desc* desc, const uint16_t* w, int64_t ro
     if (rows_per_hess < 0 || rows % rows_per_hess != 0) return IQ_ESHAPE;
     int sms = 0;
     if ((st = device_sms(&sms)) != IQ_OK) return st;
-    if (flags != nullptr && cudaMemsetAsync(flags, 0, sizeof(uint32_t), stream) != cudaSuccess) return IQ_ECUDA;
+    FlagsWord fw(flags);
+    if ((st = fw.begin(stream)) != IQ_OK) return st;
     iqk::ChoiceParams p;
     p.w = w;
     p.rows = rows;
@@ -202,9 +270,9 @@ iq_status iq_choice_search_g8(const iq_desc* desc, const uint16_t* w, int64_t ro
     p.payload = nullptr;
     p.payload_ld = 0;
     p.objective = objective;
-    p.flags = flags;
+    p.flags = fw.ptr();
     p.grid = desc->grid;
-    return launched(iqk::launch_choice_search(iqk::kChoiceIq2xsG8, p, sms, stream));
+    return fw.finish(launched(iqk::launch_choice_search(iqk::kChoiceIq2xsG8, p, sms, stream)), stream);
 }
 
 iq_status iq_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t stream) {
@@ -223,6 +291,11 @@ const char* iq_status_string(iq_status s) {
         case IQ_ESHAPE: return "invalid shape (empty, or columns not a multiple of 256)";
         case IQ_ECUDA: return "CUDA error";
         case IQ_EUNSUPPORTED: return "device is not sm_100, or the call does not take this format";
+        case IQ_ENONFINITE: return "a weight or Hessian value is NaN or infinite";
+        case IQ_EIMPORTANCE: return "an importance value is NaN, infinite or negative";
+        case IQ_ERANGE: return "a block scale overflows fp16, or a given scale is negative, infinite or NaN";
+        case IQ_ECHOICE: return "a given choice is out of the format's range";
+        case IQ_EGRID: return "a grid value lies outside the format's alphabet";
         default: return "unknown status";
     }
 }

@@ -30,11 +30,18 @@
  * they validate their arguments on the host, enqueue kernels and return. A non-IQ_OK status
  * means nothing was enqueued (except IQ_ECUDA, reported after a failed launch).
  *
- * Device-side findings (non-finite weights, bad importance, out-of-range choices, d overflowing
- * fp16, a grid value outside the format's alphabet) cannot be known on the host. The kernels OR
- * IQ_FLAG_* bits into `*flags` (a caller-owned device uint32; the call first clears it, so after
- * the stream reaches the end of the call it holds exactly this call's findings). Blocks with a
- * finding are written as the all-zero payload. `flags` may be NULL to skip reporting.
+ * Device-side findings (non-finite weights or Hessian values, bad importance, out-of-range
+ * choices, d overflowing fp16, a grid value outside the format's alphabet) cannot be known on the
+ * host. Blocks with a finding are written as the all-zero payload. How a call reports them depends
+ * on `flags`:
+ *   - flags != NULL (a caller-owned device uint32): the call stays asynchronous. It clears the word
+ *     on `stream` and the kernels OR IQ_FLAG_* bits into it, so once the stream has passed the call
+ *     the word holds exactly this call's findings; the status only covers the host-side checks.
+ *   - flags == NULL: the call is SYNCHRONOUS. The kernels report into a word the library keeps on
+ *     each device; the call waits for `stream` to finish it and returns the first finding as a
+ *     status (IQ_EGRID, IQ_ENONFINITE, IQ_EIMPORTANCE, IQ_ERANGE, IQ_ECHOICE, in that order of
+ *     precedence), so bad data never comes back as IQ_OK. Such calls on one device are serialised
+ *     by a host mutex held from clearing that word to reading it back.
  *
  * Requires an sm_100 (B200-class) device; other devices get IQ_EUNSUPPORTED.
  */
@@ -55,7 +62,13 @@ typedef enum {
     IQ_EINVAL = 1,        /* NULL pointer, unknown format, bad descriptor or stride          */
     IQ_ESHAPE = 2,        /* empty tensor, or cols not a multiple of 256 ([512, 384] case)     */
     IQ_ECUDA = 3,         /* a CUDA runtime call or kernel launch failed                       */
-    IQ_EUNSUPPORTED = 4   /* the current device is not sm_100, or the call does not take the format */
+    IQ_EUNSUPPORTED = 4,  /* the current device is not sm_100, or the call does not take the format */
+    /* device-side findings, returned only by calls made with flags == NULL (see above)          */
+    IQ_ENONFINITE = 5,    /* a weight (or, for the choice search, a Hessian value) is NaN or inf  */
+    IQ_EIMPORTANCE = 6,   /* an importance value is NaN, infinite or negative (PR #2723 review)  */
+    IQ_ERANGE = 7,        /* d rounds to fp16 infinity, or a given d is negative, infinite or NaN */
+    IQ_ECHOICE = 8,       /* a given choice is >= the format's number of choices              */
+    IQ_EGRID = 9          /* a grid value lies outside the format's alphabet                   */
 } iq_status;
 
 typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3, IQ_FMT_IQ2_S = 4 } iq_format;
@@ -67,7 +80,7 @@ typedef enum { IQ_OUT_F32 = 0, IQ_OUT_BF16 = 1 } iq_out_dtype;
 typedef enum { IQ_IN_BF16 = 0, IQ_IN_F16 = 1, IQ_IN_F32 = 2 } iq_in_dtype;
 
 /* device-side findings, ORed into *flags */
-#define IQ_FLAG_NONFINITE 1u  /* a weight is NaN or +-inf                                 */
+#define IQ_FLAG_NONFINITE 1u  /* a weight (choice search: or a Hessian value) is NaN or +-inf */
 #define IQ_FLAG_IMPORTANCE 2u /* an importance value is NaN, +-inf or negative            */
 #define IQ_FLAG_RANGE 4u      /* d rounds to fp16 infinity, or a given d is < 0, inf or NaN */
 #define IQ_FLAG_CHOICE 8u     /* a given choice is >= 16                                  */
@@ -94,10 +107,23 @@ typedef struct {
     const int8_t *grid;
     float anchor;
 } iq_desc;
+/*
+ * Two convention values are deliberately not descriptor fields:
+ *   - delta = +-1/8 (IQ1_S, IQ1_M; PR #2723, the PR #2450 worked example) belongs to the layout,
+ *     not to the encoder: a payload stores only its sign bit, and every decoder of the format
+ *     reads the value back as +-1/8. An encoder searching under another delta would write
+ *     payloads that decode to values it never scored.
+ *   - IQ1_M's anchor clamp(0.58 + 0.035 * peak_to_rms, 0.65, 0.95) is the format's own scale
+ *     predictor (PR #2513); IQ1_S's flat 0.61 is the `anchor` field's default.
+ */
 
 /* Bytes per 256-weight block: 50 (IQ1_S), 74 (IQ2_XS), 56 (IQ1_M), 82 (IQ2_S); 0 for an unknown
  * format. */
 size_t iq_block_bytes(int32_t fmt);
+
+/* Payload bytes of a [rows, cols] weight: rows * (cols / 256) * iq_block_bytes(fmt); 0 for an
+ * unknown format, a negative size or cols not a multiple of 256. */
+size_t iq_payload_bytes(int32_t fmt, int64_t rows, int64_t cols);
 
 /* Choice groups per block: 8 (IQ1_S, one per 32 weights: local scale + delta sign),
  * 16 (IQ2_XS and IQ2_S, one 4-bit local scale per 16 weights; IQ1_M, one 3-bit local scale per

@@ -20,14 +20,19 @@ def lib():
     return iq.load_library()
 
 
-def _declared_functions():
-    src = open(os.path.join(ROOT, "include", "iq.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(iq_[a-z0-9_]+)\s*\(", src)))
+def _declared_functions(header=None):
+    names = [header] if header else sorted(os.listdir(os.path.join(ROOT, "include")))
+    out = set()
+    for h in names:
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        out |= set(re.findall(r"\b(iq_[a-z0-9_]+)\s*\(", src))
+    return sorted(out)
 
 
 def test_header_declares_the_binding_symbols():
-    assert set(_declared_functions()) == set(iq.SYMBOLS)
+    assert set(_declared_functions("iq.h")) == set(iq.SYMBOLS)
+    assert set(_declared_functions("iq_probe.h")) == set(iq.PROBE_SYMBOLS)
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -48,6 +53,20 @@ def test_format_tables(lib):
         assert lib.iq_num_choices(code) == iq.CHOICES[fmt]
     assert b"sm_100a" in lib.iq_build_info()
     assert lib.iq_status_string(2).startswith(b"invalid shape")
+    for st in range(10):
+        assert lib.iq_status_string(st) != b"unknown status", st
+    assert lib.iq_status_string(10) == b"unknown status"
+    assert lib.iq_probe_fp32_ops_per_iter(0) == 8 and lib.iq_probe_fp32_ops_per_iter(3) == 16
+    assert lib.iq_probe_fp32_ops_per_iter(4) == 0
+
+
+def test_payload_bytes(lib):
+    for fmt, code in iq.IQ_FMT.items():
+        assert lib.iq_payload_bytes(code, 4096, 4096) == 4096 * 16 * iq.BLOCK_BYTES[fmt]
+        assert lib.iq_payload_bytes(code, 0, 256) == 0 and lib.iq_payload_bytes(code, 3, 0) == 0
+        assert lib.iq_payload_bytes(code, 2, 384) == 0 and lib.iq_payload_bytes(code, -1, 256) == 0
+    assert lib.iq_payload_bytes(1, 256 * 1536, 4096) == 256 * 1536 * 16 * 50
+    assert lib.iq_payload_bytes(7, 1, 256) == 0
 
 
 def _desc(fmt=1, entries=2048, grid=0x1000, anchor=0.61):
