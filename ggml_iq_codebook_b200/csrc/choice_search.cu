@@ -147,12 +147,8 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 
-#ifndef IQ_CHOICE_COLUMN_MAX_W16
-#define IQ_CHOICE_COLUMN_MAX_W16 12  // 16- and 8-column choice groups, 16 rows per CTA
-#endif
-#ifndef IQ_CHOICE_COLUMN_MAX_W32
-#define IQ_CHOICE_COLUMN_MAX_W32 0  // 32-column choice groups (IQ1_S): always tiles (measured)
-#endif
+constexpr int kColumnMaxW16 = 12;  // 16- and 8-column choice groups, 16 rows per CTA
+constexpr int kColumnMaxW32 = 0;   // 32-column choice groups (IQ1_S): always tiles (measured)
 
 template <int FMT>
 struct Cfg {
@@ -181,7 +177,7 @@ struct Cfg {
     static constexpr int oUR = oUT + W * R * 4;                   // float [R][W]: the same, by row
     static constexpr int oSw = oCurT + kBlock * R * 4;            // int [R]: row switched this step
     // update by column up to this many switched rows, else by tiles (either is bit-exact)
-    static constexpr int COLUMN_MAX = W == 32 ? IQ_CHOICE_COLUMN_MAX_W32 : IQ_CHOICE_COLUMN_MAX_W16;
+    static constexpr int COLUMN_MAX = W == 32 ? kColumnMaxW32 : kColumnMaxW16;
     static constexpr int oGrid = oSw + R * 4;                     // uint16 [E] element codes
     static constexpr int oRows = oGrid + (E * 2 + 15) / 16 * 16;  // per-row records
     static constexpr int rX = 0;                                  // bf16 [256]

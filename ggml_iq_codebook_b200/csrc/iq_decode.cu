@@ -29,20 +29,10 @@
 namespace iqk {
 namespace {
 
-#ifndef IQ_DECODE_MIN_CTAS
-#define IQ_DECODE_MIN_CTAS 1  // launch-bounds occupancy hint (CTAs per SM)
-#endif
-
-#ifndef IQ_DECODE_TILE
-#define IQ_DECODE_TILE 256  // blocks per staged payload tile
-#endif
-#ifndef IQ_DECODE_CTAS
-#define IQ_DECODE_CTAS 5  // persistent CTAs per SM
-#endif
-
 constexpr int kThreads = 256;
-constexpr int kTileBlocks = IQ_DECODE_TILE;
-constexpr int kCtasPerSm = IQ_DECODE_CTAS;
+constexpr int kMinCtas = 1;      // launch-bounds occupancy hint (CTAs per SM)
+constexpr int kTileBlocks = 256;  // blocks per staged payload tile
+constexpr int kCtasPerSm = 5;     // persistent CTAs per SM
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
@@ -205,7 +195,7 @@ __device__ __forceinline__ uint16_t grid_code(int2 raw) {
 }
 
 template <int FMT, bool BF16>
-__global__ void __launch_bounds__(kThreads, IQ_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, kMinCtas) decode_kernel(const DecodeParams p) {
     using C = DecodeCfg<FMT>;
     extern __shared__ __align__(16) char smem[];
     uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem);
