@@ -113,12 +113,17 @@ def sqrt_lognormal(shape, seed: int, device="cpu") -> torch.Tensor:
     return torch.sqrt(torch.exp(z)).to(torch.float32).to(device)
 
 
-def block_hessian(seed: int, n: int = BLOCK, offdiag_std: float = 0.02) -> torch.Tensor:
-    """H = U^-1 U^-T (fp64, symmetrised) as fp32 [n, n]."""
+def block_factor(seed: int, n: int = BLOCK, offdiag_std: float = 0.02) -> torch.Tensor:
+    """Upper-triangular U (fp64 [n, n]): diagonal uniform in [0.5, 2], above it N(0, std^2)."""
     g = torch.Generator().manual_seed(seed)
     diag = 0.5 + 1.5 * torch.rand(n, generator=g, dtype=torch.float64)
     off = offdiag_std * torch.randn((n, n), generator=g, dtype=torch.float64)
-    u = torch.triu(off, diagonal=1) + torch.diag(diag)
+    return torch.triu(off, diagonal=1) + torch.diag(diag)
+
+
+def block_hessian(seed: int, n: int = BLOCK, offdiag_std: float = 0.02) -> torch.Tensor:
+    """H = U^-1 U^-T (fp64, symmetrised) as fp32 [n, n], U = block_factor(seed)."""
+    u = block_factor(seed, n, offdiag_std)
     uinv = torch.linalg.solve_triangular(u, torch.eye(n, dtype=torch.float64), upper=True)
     h = uinv @ uinv.T
     h = 0.5 * (h + h.T)
@@ -169,6 +174,32 @@ def workload_choice_iq2xs(device="cpu", rows=4096, cols=4096):
     nblk = cols // BLOCK
     hess = torch.stack([block_hessian(5000 + b) for b in range(nblk)]).to(device)
     return {"fmt": "iq2_xs", "w": normal_bf16((rows, cols), 0.02, 1005, device), "hess": hess}
+
+
+def inverse_hessian_factor(nblk: int, seed: int = 5000, offdiag_std: float = 0.02, cross_seed: int = 7000,
+                           cross_std: float = 0.02) -> torch.Tensor:
+    """The upper Cholesky factor U of a weight's inverse Hessian (H^-1 = U^T U), fp32 [256 nblk]^2:
+    diagonal block b is block_factor(seed + b), so that block b's local Hessian U_bb^-1 U_bb^-T is
+    block_hessian(seed + b); the blocks above the diagonal are N(0, cross_std^2) (seed cross_seed),
+    the ones below it zero."""
+    n = nblk * BLOCK
+    u = torch.zeros((n, n), dtype=torch.float64)
+    g = torch.Generator().manual_seed(cross_seed)
+    for b in range(nblk):
+        s = slice(b * BLOCK, (b + 1) * BLOCK)
+        u[s, s] = block_factor(seed + b, offdiag_std=offdiag_std)
+        if b + 1 < nblk:
+            u[s, (b + 1) * BLOCK:] = cross_std * torch.randn((BLOCK, n - (b + 1) * BLOCK), generator=g,
+                                                             dtype=torch.float64)
+    return u.to(torch.float32).contiguous()
+
+
+def workload_gptq_iq2xs(device="cpu", rows=4096, cols=4096):
+    """The per-block calibration loop: the local-Hessian workload's weight and block Hessians,
+    plus the full inverse-Hessian factor U whose diagonal blocks give those Hessians."""
+    wl = workload_choice_iq2xs(device, rows, cols)
+    wl["U"] = inverse_hessian_factor(cols // BLOCK).to(device)
+    return wl
 
 
 def workload_choice_moe(device="cpu", experts=16, rows=1536, cols=4096):

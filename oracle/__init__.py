@@ -74,7 +74,9 @@ def _load(path: str | None = None):
         lib.orc_decode.restype = None
         lib.orc_decode.argtypes = [ctypes.c_int, P, P, i64, P]
         lib.orc_choice_search.restype = ctypes.c_uint32
-        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, i64, i64, i64, P, i64, P, P, P, P, P]
+        lib.orc_choice_search.argtypes = [ctypes.c_int, P, P, ctypes.c_int, i64, i64, i64, P, i64, P, P, P, P, P]
+        lib.orc_gptq_blocks.restype = ctypes.c_uint32
+        lib.orc_gptq_blocks.argtypes = [ctypes.c_int, P, ctypes.c_float, P, i64, i64, P, P, P, P, P]
         lib.orc_sqrt_diag.restype = None
         lib.orc_sqrt_diag.argtypes = [P, i64, P]
         lib.orc_f32_to_f16.restype = ctypes.c_uint16
@@ -204,7 +206,7 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
                   objective=False, return_flags=False):
     """Local-Hessian choice search over every 256-column block of w.
 
-    w: [rows, cols], or [experts, rows, cols] with hess [experts, nblk, 256, 256] (each expert's
+    w: [rows, cols] (bf16, or fp32 values), or [experts, rows, cols] with hess [experts, nblk, 256, 256] (each expert's
     rows use its own Hessian blocks); hess: [nblk, 256, 256] fp32 otherwise;
     cand: [C, (experts,) rows, nblk, B] every-choice payloads (C = 16; 8 for iq1_m).
     Returns (picks [(experts,) rows, nblk, G], payload [(experts,) rows, nblk, B]) and, with
@@ -215,7 +217,9 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     row-block with a finding gets picks 0, the all-zero payload and a NaN objective.
     Parity of the sweeps is pinned by the fp64 direct-objective replay in the tests.
     """
-    wb = _bf16_bits(w)
+    wb, kind = _weights(w)
+    if kind == IN_F16:
+        raise TypeError("the choice search takes bf16 or fp32 weights")
     lead = wb.shape[:-1]
     cols = wb.shape[-1]
     wb = wb.reshape(-1, cols)
@@ -229,7 +233,7 @@ def choice_search(fmt: str, grid: np.ndarray, w, hess: np.ndarray, cand: np.ndar
     payload = np.zeros((rows, nblk, B), dtype=np.uint8)
     tr = np.zeros((rows, nblk, 3, G), dtype=np.uint8) if trace else None
     obj = np.zeros((rows, nblk), dtype=np.float32) if objective else None
-    flags = _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
+    flags = _load().orc_choice_search(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb), kind,
                                       rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
                                       _ptr(payload), _ptr(tr), _ptr(obj))
     out = [picks.reshape(lead + (nblk, G)), payload.reshape(lead + (nblk, B))]
@@ -255,7 +259,9 @@ def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, tr
     choice_search (a row-block with a finding gets picks 8). No payload layout stores a scale per
     8 weights, so none is assembled.
     """
-    wb = _bf16_bits(w)
+    wb, kind = _weights(w)
+    if kind == IN_F16:
+        raise TypeError("the choice search takes bf16 or fp32 weights")
     lead = wb.shape[:-1]
     cols = wb.shape[-1]
     wb = wb.reshape(-1, cols)
@@ -268,7 +274,7 @@ def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, tr
     tr = np.zeros((rows, nblk, 3, 32), dtype=np.uint8) if trace else None
     obj = np.zeros((rows, nblk), dtype=np.float32) if objective else None
     flags = _load().orc_choice_search(CS_IQ2XS_G8, _ptr(np.ascontiguousarray(grid, dtype=np.int8)), _ptr(wb),
-                                      rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
+                                      kind, rows, nblk, cols, _ptr(hess), rows // nexp, _ptr(cand), _ptr(picks),
                                       None, _ptr(tr), _ptr(obj))
     out = [picks.reshape(lead + (nblk, 32))]
     if trace:
@@ -278,6 +284,28 @@ def choice_search_g8(grid: np.ndarray, w, hess: np.ndarray, cand: np.ndarray, tr
     if return_flags:
         out.append(int(flags))
     return tuple(out)
+
+
+def gptq_blocks(fmt: str, grid: np.ndarray, anchor: float, w, hess: np.ndarray, U: np.ndarray):
+    """The per-block calibration loop over one bf16 weight [rows, cols]: for each 256-column block
+    in order, the every-choice encode under sqrt(diag H_b), the local-Hessian choice search under
+    H_b, then GPTQ's propagation of the block's error E to the later columns through U (the upper
+    Cholesky factor of the inverse Hessian, [cols, cols]; hess: [cols/256, 256, 256]).
+    Returns (payload [rows, nblk, B], picks [rows, nblk, G], w_work [rows, cols] fp32: the weights
+    each block was quantised from, flags)."""
+    wb = _bf16_bits(w)
+    rows, cols = wb.shape
+    nblk = cols // 256
+    B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
+    hess = np.ascontiguousarray(hess, dtype=np.float32).reshape(nblk, 256, 256)
+    U = np.ascontiguousarray(U, dtype=np.float32).reshape(cols, cols)
+    payload = np.zeros((rows, nblk, B), dtype=np.uint8)
+    picks = np.zeros((rows, nblk, G), dtype=np.uint8)
+    w_work = np.zeros((rows, cols), dtype=np.float32)
+    flags = _load().orc_gptq_blocks(FMT[fmt], _ptr(np.ascontiguousarray(grid, dtype=np.int8)), float(anchor),
+                                    _ptr(wb), rows, cols, _ptr(hess), _ptr(U), _ptr(payload), _ptr(picks),
+                                    _ptr(w_work))
+    return payload, picks, w_work, int(flags)
 
 
 def sqrt_diag(hess: np.ndarray) -> np.ndarray:
