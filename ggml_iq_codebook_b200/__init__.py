@@ -34,7 +34,8 @@ IQ_IN = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
 
 SYMBOLS = ("iq_block_bytes", "iq_payload_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
-           "iq_choice_search", "iq_choice_search_g8", "iq_sqrt_diag", "iq_status_string", "iq_build_info")
+           "iq_choice_search", "iq_choice_search_g8", "iq_gptq_workspace_bytes", "iq_gptq_blocks", "iq_sqrt_diag",
+           "iq_status_string", "iq_build_info")
 PROBE_SYMBOLS = ("iq_probe_fp32", "iq_probe_fp32_ops_per_iter")  # include/iq_probe.h: measurement only
 
 
@@ -77,6 +78,11 @@ def load_library(path: str = LIB_PATH):
                                      P]
     lib.iq_choice_search_g8.restype = ctypes.c_int
     lib.iq_choice_search_g8.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, i64, P, i64, i64, P, P, P, P]
+    lib.iq_gptq_workspace_bytes.restype = ctypes.c_size_t
+    lib.iq_gptq_workspace_bytes.argtypes = [i32, i64]
+    lib.iq_gptq_blocks.restype = ctypes.c_int
+    lib.iq_gptq_blocks.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, P, i64, P, ctypes.c_size_t, P, P, P,
+                                   P, P]
     lib.iq_sqrt_diag.restype = ctypes.c_int
     lib.iq_sqrt_diag.argtypes = [P, i64, P, P]
     lib.iq_status_string.restype = ctypes.c_char_p
@@ -327,6 +333,59 @@ def iq_choice_search_g8(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, cand:
                                    None if objective is None else objective.data_ptr(),
                                    None if flags is None else flags.data_ptr(), _stream(stream)))
     return picks
+
+
+def iq_gptq_workspace_bytes(fmt: str, rows: int) -> int:
+    return int(load_library().iq_gptq_workspace_bytes(IQ_FMT[fmt], rows))
+
+
+def iq_gptq_blocks(desc: IQDesc, w: torch.Tensor, hess: torch.Tensor, U: torch.Tensor,
+                   workspace: torch.Tensor | None = None, payload: torch.Tensor | None = None,
+                   picks: torch.Tensor | None = None, w_work: torch.Tensor | None = None,
+                   flags: torch.Tensor | None = None, stream=None):
+    """The per-block calibration loop over one bf16 weight [rows, cols] in one call: for each
+    256-column block in order, the every-choice encode under sqrt(diag H_b), the local-Hessian
+    choice search under H_b, and GPTQ's propagation of the block's error to the later columns
+    through U (fp32 [cols, cols] upper-triangular factor of the inverse Hessian; hess fp32
+    [cols/256, 256, 256]). workspace: uint8 CUDA tensor of iq_gptq_workspace_bytes(fmt, rows)
+    bytes (allocated here if omitted). Returns (payload uint8 [rows, cols/256, B], picks uint8
+    [rows, cols/256, G], w_work fp32 [rows, cols]: the weights each block was quantised from)."""
+    lib = load_library()
+    fmt = _fmt_of(desc)
+    _need(w, torch.bfloat16, "w")
+    _need(hess, torch.float32, "hess")
+    _need(U, torch.float32, "U")
+    if w.dim() != 2 or w.stride(-1) != 1:
+        raise IQError("w must be [rows, cols] with a contiguous last dim")
+    rows, cols = w.shape
+    if cols == 0 or cols % 256:
+        raise IQError(f"w must have a positive multiple of 256 columns, got {cols}")
+    nblk = cols // 256
+    if not hess.is_contiguous() or hess.numel() != nblk * 256 * 256:
+        raise IQError("hess must be contiguous [cols/256, 256, 256]")
+    if U.dim() != 2 or U.shape[0] != cols or U.shape[1] < cols or U.stride(-1) != 1:
+        raise IQError("U must be [cols, >= cols] with a contiguous last dim")
+    B, G = BLOCK_BYTES[fmt], CHOICE_GROUPS[fmt]
+    need = iq_gptq_workspace_bytes(fmt, rows)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=w.device)
+    elif workspace.dtype != torch.uint8 or workspace.numel() < need or not workspace.is_contiguous():
+        raise IQError(f"workspace must be a contiguous uint8 tensor of at least {need} bytes")
+    if payload is None:
+        payload = torch.empty((rows, nblk, B), dtype=torch.uint8, device=w.device)
+    if picks is None:
+        picks = torch.empty((rows, nblk, G), dtype=torch.uint8, device=w.device)
+    if w_work is None:
+        w_work = torch.empty((rows, cols), dtype=torch.float32, device=w.device)
+    for t, shape, dt, name in ((payload, (rows, nblk, B), torch.uint8, "payload"), (picks, (rows, nblk, G), torch.uint8,
+                               "picks"), (w_work, (rows, cols), torch.float32, "w_work")):
+        if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous():
+            raise IQError(f"{name} must be a contiguous {dt} tensor of shape {shape}")
+    _check(lib.iq_gptq_blocks(ctypes.byref(desc), w.data_ptr(), rows, cols, w.stride(0), hess.data_ptr(),
+                              U.data_ptr(), U.stride(0), workspace.data_ptr(), workspace.numel(), payload.data_ptr(),
+                              picks.data_ptr(), w_work.data_ptr(), None if flags is None else flags.data_ptr(),
+                              _stream(stream)))
+    return payload, picks, w_work
 
 
 def iq_sqrt_diag(hess: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

@@ -221,9 +221,14 @@ iq_status iq_choice_search(const iq_desc* desc, const uint16_t* w, int64_t rows,
     if ((st = fw.begin(stream)) != IQ_OK) return st;
     iqk::ChoiceParams p;
     p.w = w;
+    p.w_f32 = 0;
     p.rows = rows;
     p.nblk = nblk;
     p.ldw = ldw;
+    p.blk0 = 0;
+    p.nblk_run = nblk;
+    p.cand_blk0 = 0;
+    p.delta_out = nullptr;
     p.hess = hess;
     p.rows_per_hess = rows_per_hess;
     p.cand = cand;
@@ -258,9 +263,14 @@ iq_status iq_choice_search_g8(const iq_desc* desc, const uint16_t* w, int64_t ro
     if ((st = fw.begin(stream)) != IQ_OK) return st;
     iqk::ChoiceParams p;
     p.w = w;
+    p.w_f32 = 0;
     p.rows = rows;
     p.nblk = nblk;
     p.ldw = ldw;
+    p.blk0 = 0;
+    p.nblk_run = nblk;
+    p.cand_blk0 = 0;
+    p.delta_out = nullptr;
     p.hess = hess;
     p.rows_per_hess = rows_per_hess;
     p.cand = cand + iqk::kChoiceG8FirstLs * cand_choice_stride;  // the candidate for ls = 8
@@ -273,6 +283,110 @@ iq_status iq_choice_search_g8(const iq_desc* desc, const uint16_t* w, int64_t ro
     p.flags = fw.ptr();
     p.grid = desc->grid;
     return fw.finish(launched(iqk::launch_choice_search(iqk::kChoiceIq2xsG8, p, sms, stream)), stream);
+}
+
+namespace {
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+}  // namespace
+
+size_t iq_gptq_workspace_bytes(int32_t fmt, int64_t rows) {
+    const size_t b = iq_block_bytes(fmt), c = static_cast<size_t>(iq_num_choices(fmt));
+    if (b == 0 || rows <= 0) return 0;
+    const size_t r = static_cast<size_t>(rows);
+    return round256(256 * sizeof(float)) + round256(c * r * b) + round256(r * 256 * sizeof(float));
+}
+
+iq_status iq_gptq_blocks(const iq_desc* desc, const uint16_t* w, int64_t rows, int64_t cols, int64_t ldw,
+                         const float* hess, const float* U, int64_t ldu, void* workspace, size_t workspace_bytes,
+                         uint8_t* payload, uint8_t* picks, float* w_work, uint32_t* flags, cudaStream_t stream) {
+    iq_status st = check_desc(desc);
+    if (st != IQ_OK) return st;
+    if (w == nullptr || hess == nullptr || U == nullptr || workspace == nullptr || payload == nullptr ||
+        picks == nullptr || w_work == nullptr)
+        return IQ_EINVAL;
+    if (rows <= 0 || cols <= 0 || cols % 256 != 0) return IQ_ESHAPE;
+    if (ldw < cols || ldw % 8 != 0 || !aligned(w, 16) || !aligned(hess, 16)) return IQ_EINVAL;
+    if (ldu < cols || ldu % 4 != 0 || !aligned(U, 16) || !aligned(w_work, 16) || !aligned(payload, 2)) return IQ_EINVAL;
+    if (!aligned(workspace, 256) || workspace_bytes < iq_gptq_workspace_bytes(desc->fmt, rows)) return IQ_EINVAL;
+    int sms = 0;
+    if ((st = device_sms(&sms)) != IQ_OK) return st;
+    FlagsWord fw(flags);
+    if ((st = fw.begin(stream)) != IQ_OK) return st;
+
+    const int64_t nblk = cols / 256, B = static_cast<int64_t>(iq_block_bytes(desc->fmt));
+    char* ws = static_cast<char*>(workspace);
+    float* imp = reinterpret_cast<float*>(ws);
+    uint8_t* cand = reinterpret_cast<uint8_t*>(ws + round256(256 * sizeof(float)));
+    float* e = reinterpret_cast<float*>(ws + round256(256 * sizeof(float)) +
+                                        round256(static_cast<size_t>(iq_num_choices(desc->fmt)) * rows * B));
+    const bool iq2 = desc->fmt == IQ_FMT_IQ2_XS || desc->fmt == IQ_FMT_IQ2_S;
+
+    cudaError_t err = iqk::launch_bf16_to_f32(w, rows, cols, ldw, w_work, stream);
+    for (int64_t b = 0; b < nblk && err == cudaSuccess; ++b) {
+        const int64_t o = 256 * b;
+        // the block's candidates: the every-choice encode of the compensated weights under
+        // sqrt(diag H_b)
+        err = iqk::launch_sqrt_diag(hess + o * 256, 1, imp, stream);
+        if (err != cudaSuccess) break;
+        iqk::EncodeParams ep;
+        ep.w = w_work + o;
+        ep.w_dtype = IQ_IN_F32;
+        ep.rows = rows;
+        ep.nblk = 1;
+        ep.ldw = cols;
+        ep.w_bstride = 0;
+        ep.imp = imp;
+        ep.imp_bstride = 0;
+        ep.choices = nullptr;
+        ep.scales = nullptr;
+        ep.scales_stride = 0;
+        ep.payload = cand;
+        ep.flags = fw.ptr();
+        ep.grid = desc->grid;
+        ep.anchor = desc->anchor;
+        ep.nb = rows;
+        err = iq2 ? iqk::launch_iq2_encode(desc->fmt, ep, iqk::kEvery, sms, stream)
+                  : iqk::launch_iq1_encode(desc->fmt, ep, iqk::kEvery, sms, stream);
+        if (err != cudaSuccess) break;
+        // the local-Hessian search of block b, which also leaves the block's final Delta in e
+        iqk::ChoiceParams cp;
+        cp.w = w_work;
+        cp.w_f32 = 1;
+        cp.rows = rows;
+        cp.nblk = nblk;
+        cp.ldw = cols;
+        cp.blk0 = b;
+        cp.nblk_run = 1;
+        cp.cand_blk0 = b;
+        cp.hess = hess;
+        cp.rows_per_hess = rows;
+        cp.cand = cand;
+        cp.cand_ld = 1;
+        cp.cand_cstride = rows * B;
+        cp.picks = picks;
+        cp.payload = payload;
+        cp.payload_ld = nblk;
+        cp.objective = nullptr;
+        cp.delta_out = e;
+        cp.flags = fw.ptr();
+        cp.grid = desc->grid;
+        err = iqk::launch_choice_search(desc->fmt, cp, sms, stream);
+        if (err != cudaSuccess || b + 1 == nblk) break;
+        // GPTQ's compensation of the later columns
+        err = iqk::launch_gptq_solve(e, U + o * ldu + o, ldu, rows, stream);
+        if (err != cudaSuccess) break;
+        iqk::GptqUpdateParams up;
+        up.w = w_work;
+        up.y = e;
+        up.u = U + o * ldu;
+        up.rows = rows;
+        up.ldw = cols;
+        up.ldu = ldu;
+        up.col0 = o + 256;
+        up.ncols = cols - o - 256;
+        err = iqk::launch_gptq_update(up, sms, stream);
+    }
+    return fw.finish(launched(err), stream);
 }
 
 iq_status iq_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t stream) {

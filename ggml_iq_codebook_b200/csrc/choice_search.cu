@@ -170,23 +170,23 @@ struct Cfg {
     static constexpr int WO = W / SPLIT;                        // group columns per lane
     static constexpr int BPAD = (kChoices * B + 15) / 16 * 16;  // candidate bytes per row
     // shared memory layout (bytes)
-    static constexpr int oHp = 0;                                 // float [2][W][256], double buffer
-    static constexpr int oCurT = oHp + 2 * W * kBlock * 4;        // float [256][R], step 2 only
-    // the sweeps' u of the rows that switched, in the curT area (free once step 2 is done)
-    static constexpr int oUT = oCurT;                             // float [W][R]
-    static constexpr int oUR = oUT + W * R * 4;                   // float [R][W]: the same, by row
-    static constexpr int oSw = oCurT + kBlock * R * 4;            // int [R]: row switched this step
+    static constexpr int oHp = 0;                             // float [2][W][256], double buffer
+    static constexpr int oCurT = oHp + 2 * W * kBlock * 4;    // float [256][R]: the rows' current Delta
+    static constexpr int oUT = oCurT + kBlock * R * 4;        // float [W][R]: u of the rows that switched
+    static constexpr int oUR = oUT + W * R * 4;               // float [R][W]: the same, by row
+    static constexpr int oT2 = oUR + R * W * 4;               // float [R][G][NC]: u^T H_gg u per candidate
+    static constexpr int oSw = oT2 + R * G * NC * 4;          // int [R]: row switched this step
     // update by column up to this many switched rows, else by tiles (either is bit-exact)
     static constexpr int COLUMN_MAX = W == 32 ? kColumnMaxW32 : kColumnMaxW16;
     static constexpr int oGrid = oSw + R * 4;                     // uint16 [E] element codes
     static constexpr int oRows = oGrid + (E * 2 + 15) / 16 * 16;  // per-row records
-    static constexpr int rX = 0;                                  // bf16 [256]
-    static constexpr int rCur = rX + kBlock * 2;                  // float [256]
-    static constexpr int rGrad = rCur + kBlock * 4;               // float [256]
+    static constexpr int rGrad = 0;                               // float [256]
     static constexpr int rPick = rGrad + kBlock * 4;              // int [G]
     static constexpr int rCand = (rPick + G * 4 + 15) / 16 * 16;  // uint8 [16][B]
     static constexpr int rBytes = (rCand + BPAD + 15) / 16 * 16;
     static constexpr int smem = oRows + R * rBytes;
+    // two CTAs share an SM (228 KiB of shared memory, 1 KiB reserved per CTA)
+    static_assert(2 * (smem + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 // Pairwise tree over N values: (p0 + p1), (p2 + p3), ... then up, as the oracle sums.
@@ -212,22 +212,53 @@ __device__ __forceinline__ void half_argmin(float v, int c, unsigned mask, float
     cbest = c;
 }
 
-// v[i] = sum over k < W (fma chain, k ascending) of Hp[k][col0 + i] * a[k], for NO columns.
-// The next panel row is loaded while the current one is used (software pipelining).
+// v[i] = sum over k < W (fma chain, k ascending, starting from the product) of
+// Hp[k][col0 + i] * a[k], for NO columns. Adjacent columns run as one packed fma.rn.f32x2 (two
+// independent IEEE fmas, so every chain rounds exactly as the scalar one); the next panel row is
+// loaded while the current one is used.
 template <int W, int NO>
 __device__ __forceinline__ void group_matvec(const float* Hp, int col0, const float a[W], float v[NO]) {
+    static_assert(NO % 4 == 0, "16-byte panel reads");
     float h[NO], hn[NO];
+    float2 acc[NO / 2];
     load_vec<NO>(Hp + col0, h);
     load_vec<NO>(Hp + kBlock + col0, hn);
+    {
+        const float2 a0 = make_float2(a[0], a[0]);
 #pragma unroll
-    for (int i = 0; i < NO; ++i) v[i] = __fmul_rn(h[i], a[0]);
+        for (int t = 0; t < NO / 2; ++t) acc[t] = __fmul2_rn(make_float2(h[2 * t], h[2 * t + 1]), a0);
+    }
 #pragma unroll
     for (int k = 1; k < W; ++k) {
 #pragma unroll
         for (int i = 0; i < NO; ++i) h[i] = hn[i];
         if (k + 1 < W) load_vec<NO>(Hp + (k + 1) * kBlock + col0, hn);
+        const float2 ak = make_float2(a[k], a[k]);
 #pragma unroll
-        for (int i = 0; i < NO; ++i) v[i] = __fmaf_rn(h[i], a[k], v[i]);
+        for (int t = 0; t < NO / 2; ++t) acc[t] = __ffma2_rn(make_float2(h[2 * t], h[2 * t + 1]), ak, acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < NO / 2; ++t) {
+        v[2 * t] = acc[t].x;
+        v[2 * t + 1] = acc[t].y;
+    }
+}
+
+// A 4-row x 4-column register tile of gradient chains: acc[r][c] = fma(h[c], x[r], acc[r][c]) for
+// one k, as two packed fmas per row (the pairs are two independent columns).
+__device__ __forceinline__ void tile_fma(float2 acc[4][2], const float4 hv, const float4 xv, bool first) {
+    const float2 h01 = make_float2(hv.x, hv.y), h23 = make_float2(hv.z, hv.w);
+    const float xr[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        const float2 x2 = make_float2(xr[rr], xr[rr]);
+        if (first) {
+            acc[rr][0] = __fmul2_rn(h01, x2);
+            acc[rr][1] = __fmul2_rn(h23, x2);
+        } else {
+            acc[rr][0] = __ffma2_rn(h01, x2, acc[rr][0]);
+            acc[rr][1] = __ffma2_rn(h23, x2, acc[rr][1]);
+        }
     }
 }
 
@@ -244,13 +275,48 @@ __device__ __forceinline__ float join_parts(float t, unsigned mask) {
     return SPLIT == 1 ? t : __fadd_rn(t, __shfl_xor_sync(mask, t, NC));
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const ChoiceParams p) {
+// u^T H_gg u over this lane's candidate: (H_gg u) for this lane's columns, the products with u,
+// and the pairwise tree over the group's W columns (joined across the lanes of a candidate).
+template <int W, int WO, int SPLIT, int NC>
+__device__ __forceinline__ float quad_form(const float* Hp, int g, int part, const float u[W], unsigned mask) {
+    float v[WO], up[WO];
+    group_matvec<W, WO>(Hp, g * W + part * WO, u, v);
+    lane_part<W, WO>(u, part, up);
+#pragma unroll
+    for (int i = 0; i < WO; ++i) v[i] = __fmul_rn(up[i], v[i]);
+    return join_parts<SPLIT, NC>(tree_sum<WO>(v), mask);
+}
+
+// Whether a staged grid row lies in the candidates' alphabet ({-1, 0, 1} or {1, 3, 5, 7}).
+template <int DF>
+__device__ __forceinline__ bool grid_row_ok(int2 raw) {
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
+        ok &= (DF == IQ_FMT_IQ1_S || DF == IQ_FMT_IQ1_M) ? (v >= -1 && v <= 1) : (v == 1 || v == 3 || v == 5 || v == 7);
+    }
+    return ok;
+}
+
+// Eight consecutive weights of a row as fp32 (exact): bf16 bits, or fp32 values.
+template <bool F32>
+__device__ __forceinline__ void load_x8(const void* xrow, int i8, float xv[8]) {
+    if (F32) {
+        const float4* q = reinterpret_cast<const float4*>(xrow) + 2 * i8;
+        const float4 a = __ldg(q), b = __ldg(q + 1);
+        xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w; xv[4] = b.x; xv[5] = b.y; xv[6] = b.z; xv[7] = b.w;
+    } else {
+        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(xrow) + i8), xv);
+    }
+}
+
+template <int FMT, bool F32>
+__global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const ChoiceParams p) {
     using C = Cfg<FMT>;
-    constexpr int W = C::W, G = C::G, kRows = C::R, kThreads = C::T, WO = C::WO;
-    static_assert(C::SPLIT * C::NC == kChoices && (W & (W - 1)) == 0, "halves join as the tree's last level");
+    constexpr int W = C::W, G = C::G, kRows = C::R, kThreads = C::T, WO = C::WO, NC = C::NC;
+    static_assert(C::SPLIT * NC == kChoices && (W & (W - 1)) == 0, "halves join as the tree's last level");
     static_assert(kThreads == C::RG * 64, "gradient tiles: 4 rows x 4 columns per thread");
-    static_assert(2 * W * kRows <= kBlock * kRows, "u buffers fit in the curT area");
     extern __shared__ __align__(16) char smem[];
     float* curT = reinterpret_cast<float*>(smem + C::oCurT);
     float* uT = reinterpret_cast<float*>(smem + C::oUT);
@@ -262,22 +328,24 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     // share one Hessian block are adjacent in launch order.
     const int64_t nexp = p.rows / p.rows_per_hess;
     const int64_t tiles_e = (p.rows_per_hess + kRows - 1) / kRows;
-    const int64_t blk = blockIdx.x / (nexp * tiles_e);
-    const int64_t rem = blockIdx.x - blk * nexp * tiles_e;
+    const int64_t blk_rel = blockIdx.x / (nexp * tiles_e);
+    const int64_t blk = p.blk0 + blk_rel;
+    const int64_t rem = blockIdx.x - blk_rel * nexp * tiles_e;
     const int64_t expert = rem / tiles_e;
     const int64_t tile_row0 = (rem - expert * tiles_e) * kRows;
     const int tid = threadIdx.x, hr = tid >> 4, c = tid & 15;
-    const int ch = c % C::NC, part = c / C::NC;  // this lane's candidate, and its half of the columns
+    const int ch = c % NC, part = c / NC;  // this lane's candidate, and its half of the columns
     const unsigned hmask = 0xFFFFu << (16 * (hr & 1));  // this half-warp's lanes within the warp
     const int64_t row = expert * p.rows_per_hess + tile_row0 + hr;
     const bool active = tile_row0 + hr < p.rows_per_hess;
     char* rec = smem + C::oRows + hr * C::rBytes;
-    uint16_t* xb = reinterpret_cast<uint16_t*>(rec + C::rX);
-    float* cur = reinterpret_cast<float*>(rec + C::rCur);
     float* grad = reinterpret_cast<float*>(rec + C::rGrad);
     int* pick = reinterpret_cast<int*>(rec + C::rPick);
     uint8_t* cand = reinterpret_cast<uint8_t*>(rec + C::rCand);
+    float* t2row = reinterpret_cast<float*>(smem + C::oT2) + hr * G * NC;  // [G][NC]
     const float* H = p.hess + (expert * p.nblk + blk) * kBlock * kBlock;
+    const void* xrow = F32 ? static_cast<const void*>(static_cast<const float*>(p.w) + row * p.ldw + blk * kBlock)
+                           : static_cast<const void*>(static_cast<const uint16_t*>(p.w) + row * p.ldw + blk * kBlock);
 
     // H panels (the W rows of one choice group) stream through a double buffer: step s of the
     // 3G group steps (step 2, then two sweeps) uses panel s % G from buffer s & 1.
@@ -290,27 +358,30 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
     };
     prefetch(0);
 
-    // ---- stage the grid codes, the row's x (bf16) and its candidate payloads (lanes past the
-    // format's NC candidates stage zeros and never win)
-    for (int q = tid; q < C::E; q += kThreads) sgrid[q] = grid_code<C::DF>(__ldg(reinterpret_cast<const int2*>(p.grid) + q));
+    // ---- stage the grid codes (checking the alphabet) and the row's candidate payloads (lanes
+    // past the format's NC candidates stage zeros and never win); a non-finite weight taints the row
+    bool grid_bad = false, h_bad = false, row_bad = false;
+    for (int q = tid; q < C::E; q += kThreads) {
+        const int2 raw = __ldg(reinterpret_cast<const int2*>(p.grid) + q);
+        sgrid[q] = grid_code<C::DF>(raw);
+        grid_bad |= !grid_row_ok<C::DF>(raw);
+    }
     if (active) {
-        const uint4* xs = reinterpret_cast<const uint4*>(p.w + row * p.ldw + blk * kBlock);
         bool nonfinite = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-            const uint4 v = __ldg(xs + 2 * c + t);
-            reinterpret_cast<uint4*>(xb)[2 * c + t] = v;
             float xv[8];
-            unpack8_bf16(v, xv);
+            load_x8<F32>(xrow, 2 * c + t, xv);
 #pragma unroll
             for (int j = 0; j < 8; ++j) nonfinite |= !isfinite(xv[j]);
         }
-        if (__any_sync(hmask, nonfinite) && c == 0) raise_flags(p.flags, IQ_FLAG_NONFINITE);
+        row_bad = __any_sync(hmask, nonfinite);
         // 2-byte copies (B is even and the caller's candidates are 2-byte aligned), all loads
         // issued before the stores
         uint16_t* dst = reinterpret_cast<uint16_t*>(cand + c * C::B);
         if (c < C::NC) {
-            const uint16_t* src = reinterpret_cast<const uint16_t*>(p.cand + c * p.cand_cstride + (row * p.cand_ld + blk) * C::B);
+            const uint16_t* src = reinterpret_cast<const uint16_t*>(
+                p.cand + c * p.cand_cstride + (row * p.cand_ld + (blk - p.cand_blk0)) * C::B);
             uint16_t stage[C::B / 2];
 #pragma unroll
             for (int i = 0; i < C::B / 2; ++i) stage[i] = __ldg(src + i);
@@ -332,7 +403,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
             // decode8 takes the format's own choice group: for 8-column groups, the 16-column
             // group that holds the scale nibble
             decode8<C::DF>(cand + ch * C::B, sgrid, C::G8 ? (g >> 1) : g, (g * W + 8 * t) >> 3, xh);
-            unpack8_bf16(reinterpret_cast<const uint4*>(xb)[(g * W) / 8 + t], xv);
+            load_x8<F32>(xrow, (g * W) / 8 + t, xv);
 #pragma unroll
             for (int j = 0; j < 8; ++j) dl[8 * t + j] = __fsub_rn(xv[j], xh[j]);
         }
@@ -344,41 +415,38 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         return reinterpret_cast<float*>(smem + C::oRows + r * C::rBytes + C::rGrad);
     };
 
-    // ---- step 2 (own diagonal block) fused with the initial gradient grad = H Delta
-    float gacc[4][4];
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) gacc[rr][cc] = 0.0f;
+    // ---- step 2 (each group's own diagonal block), fused with the initial gradient grad = H Delta
+    // and with the first sweep's curvature terms: u = Delta(c) - Delta(pick) changes only when
+    // group g itself switches, so u^T H_gg u is scored here, once, while panel g is resident.
+    float2 gacc[4][2];
     for (int g = 0; g < G; ++g) {
         cp_async_wait_all();
         __syncthreads();  // panel g has landed; every thread is done with the other buffer
         prefetch(g + 1);
         const float* Hp = panel(g);
+        // this thread's 16-byte chunks of the panel it staged must be finite
+        for (int i = tid; i < W * kBlock / 4; i += kThreads) {
+            const float4 v = reinterpret_cast<const float4*>(Hp)[i];
+            h_bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+        }
         if (active) {
-            float dl[W], v[WO];
+            float dl[W];
             delta_of(g, dl);
-            group_matvec<W, WO>(Hp, g * W + part * WO, dl, v);
-            {
-                float dp[WO];
-                lane_part<W, WO>(dl, part, dp);
-#pragma unroll
-                for (int i = 0; i < WO; ++i) v[i] = __fmul_rn(dp[i], v[i]);
-            }
-            const float t = join_parts<C::SPLIT, C::NC>(tree_sum<WO>(v), hmask);
-            const float score = c < C::NC ? t : INFINITY;
+            const float sq = quad_form<W, WO, C::SPLIT, NC>(Hp, g, part, dl, hmask);  // every lane joins
+            const float score = c < NC ? sq : INFINITY;
             float best;
             int cstar;
             half_argmin(score, c, hmask, best, cstar);
             if (c == cstar) {
 #pragma unroll
-                for (int i = 0; i < W; i += 4) {
-                    *reinterpret_cast<float4*>(cur + g * W + i) = make_float4(dl[i], dl[i + 1], dl[i + 2], dl[i + 3]);
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) curT[(g * W + i + t) * kRows + hr] = dl[i + t];
-                }
+                for (int i = 0; i < W; ++i) curT[(g * W + i) * kRows + hr] = dl[i];
                 pick[g] = c;
             }
+            // the winner's Delta by shuffles, then u = Delta(c) - Delta(pick) in place
+#pragma unroll
+            for (int i = 0; i < W; ++i) dl[i] = __fsub_rn(dl[i], __shfl_sync(hmask, dl[i], cstar, 16));
+            const float t2 = quad_form<W, WO, C::SPLIT, NC>(Hp, g, part, dl, hmask);
+            if (part == 0) t2row[g * NC + ch] = t2;
         }
         __syncthreads();
         // grad_i += H[k][i] cur_k over this group's k: a 4-row x 4-column tile per thread, fed by
@@ -387,27 +455,22 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         for (int k = 0; k < W; ++k) {
             const float4 cv = *reinterpret_cast<const float4*>(curT + (g * W + k) * kRows + 4 * rg);
             const float4 hv = *reinterpret_cast<const float4*>(Hp + k * kBlock + 4 * cg);
-            const float cr[4] = {cv.x, cv.y, cv.z, cv.w}, hc[4] = {hv.x, hv.y, hv.z, hv.w};
-            if (g == 0 && k == 0) {
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) gacc[rr][cc] = __fmul_rn(hc[cc], cr[rr]);
-            } else {
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) gacc[rr][cc] = __fmaf_rn(hc[cc], cr[rr], gacc[rr][cc]);
-            }
+            tile_fma(gacc, hv, cv, g == 0 && k == 0);
         }
     }
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr)
         *reinterpret_cast<float4*>(grad_row(4 * rg + rr) + 4 * cg) =
-            make_float4(gacc[rr][0], gacc[rr][1], gacc[rr][2], gacc[rr][3]);
+            make_float4(gacc[rr][0].x, gacc[rr][0].y, gacc[rr][1].x, gacc[rr][1].y);
+    grid_bad = __syncthreads_or(grid_bad);
+    h_bad = __syncthreads_or(h_bad);
+    if (tid == 0) raise_flags(p.flags, (grid_bad ? IQ_FLAG_GRID : 0u) | (h_bad ? IQ_FLAG_NONFINITE : 0u));
+    if (active && c == 0 && row_bad) raise_flags(p.flags, IQ_FLAG_NONFINITE);
 
-    // ---- step 3: two sweeps over the groups. Each row decides (lane per choice); then every
-    // thread updates its gradient tile for the rows that switched.
+    // ---- step 3: two sweeps over the groups. Each row decides (lane per choice) from the stored
+    // curvature term and the current gradient; a row that switches in the first sweep rescores
+    // that group's curvature terms around its new pick for the second. Then every thread
+    // updates its gradient tile for the rows that switched.
     for (int step = G; step < 3 * G; ++step) {
         const int g = step % G;
         cp_async_wait_all();
@@ -416,43 +479,41 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
         const float* Hp = panel(step);
         int switched = 0;
         if (active) {
-            float dl[W], u[W], v[WO];
+            float dl[W], u[W];
             delta_of(g, dl);
-            {
-                float cgv[W];
-                load_vec<W>(cur + g * W, cgv);
 #pragma unroll
-                for (int i = 0; i < W; ++i) u[i] = __fsub_rn(dl[i], cgv[i]);
-            }
-            group_matvec<W, WO>(Hp, g * W + part * WO, u, v);
+            for (int i = 0; i < W; ++i) u[i] = __fsub_rn(dl[i], curT[(g * W + i) * kRows + hr]);
             float gain;
             {
                 float gq[WO], p1[WO], up[WO];
                 load_vec<WO>(grad + g * W + part * WO, gq);
                 lane_part<W, WO>(u, part, up);
 #pragma unroll
-                for (int i = 0; i < WO; ++i) {
-                    p1[i] = __fmul_rn(up[i], gq[i]);
-                    v[i] = __fmul_rn(up[i], v[i]);
-                }
-                const float t1 = join_parts<C::SPLIT, C::NC>(tree_sum<WO>(p1), hmask);
-                const float t2 = join_parts<C::SPLIT, C::NC>(tree_sum<WO>(v), hmask);
-                gain = c < C::NC ? __fmaf_rn(2.0f, t1, t2) : INFINITY;
+                for (int i = 0; i < WO; ++i) p1[i] = __fmul_rn(up[i], gq[i]);
+                const float t1 = join_parts<C::SPLIT, NC>(tree_sum<WO>(p1), hmask);
+                gain = c < NC ? __fmaf_rn(2.0f, t1, t2row[g * NC + ch]) : INFINITY;
             }
             float best;
             int cstar;
             half_argmin(gain, c, hmask, best, cstar);
             switched = best < 0.0f;  // uniform over the half-warp
-            if (switched && c == cstar) {
+            if (switched) {
+                if (c == cstar) {
 #pragma unroll
-                for (int i = 0; i < W; ++i) uT[i * kRows + hr] = u[i];
+                    for (int i = 0; i < W; ++i) uT[i * kRows + hr] = u[i];
 #pragma unroll
-                for (int i = 0; i < W; i += 4)
-                    *reinterpret_cast<float4*>(uR + hr * W + i) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
+                    for (int i = 0; i < W; i += 4)
+                        *reinterpret_cast<float4*>(uR + hr * W + i) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
 #pragma unroll
-                for (int i = 0; i < W; i += 4)
-                    *reinterpret_cast<float4*>(cur + g * W + i) = make_float4(dl[i], dl[i + 1], dl[i + 2], dl[i + 3]);
-                pick[g] = c;
+                    for (int i = 0; i < W; ++i) curT[(g * W + i) * kRows + hr] = dl[i];
+                    pick[g] = c;
+                }
+                if (step < 2 * G) {  // the second sweep's curvature terms around the new pick
+#pragma unroll
+                    for (int i = 0; i < W; ++i) dl[i] = __fsub_rn(dl[i], __shfl_sync(hmask, dl[i], cstar, 16));
+                    const float t2 = quad_form<W, WO, C::SPLIT, NC>(Hp, g, part, dl, hmask);
+                    if (part == 0) t2row[g * NC + ch] = t2;
+                }
             }
         }
         if (c == 0) swf[hr] = switched;
@@ -482,48 +543,65 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
                 }
             }
         } else if (swmask != 0 && ((swmask >> (4 * rg)) & 15u) != 0) {
-            float acc[4][4];
+            float2 acc[4][2];
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
                 const float4 a = *reinterpret_cast<const float4*>(grad_row(4 * rg + rr) + 4 * cg);
-                acc[rr][0] = a.x; acc[rr][1] = a.y; acc[rr][2] = a.z; acc[rr][3] = a.w;
+                acc[rr][0] = make_float2(a.x, a.y);
+                acc[rr][1] = make_float2(a.z, a.w);
             }
 #pragma unroll 4
             for (int k = 0; k < W; ++k) {
                 const float4 uv = *reinterpret_cast<const float4*>(uT + k * kRows + 4 * rg);
                 const float4 hv = *reinterpret_cast<const float4*>(Hp + k * kBlock + 4 * cg);
-                const float ur[4] = {uv.x, uv.y, uv.z, uv.w}, hc[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) acc[rr][cc] = __fmaf_rn(hc[cc], ur[rr], acc[rr][cc]);
+                tile_fma(acc, hv, uv, false);
             }
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr)
                 if ((swmask >> (4 * rg + rr)) & 1u)  // rows that kept their choice keep their gradient
                     *reinterpret_cast<float4*>(grad_row(4 * rg + rr) + 4 * cg) =
-                        make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+                        make_float4(acc[rr][0].x, acc[rr][0].y, acc[rr][1].x, acc[rr][1].y);
         }
     }
 
     __syncthreads();  // every gradient update has landed
+    // A row-block with a finding (a non-finite weight in the row, a non-finite entry in its
+    // Hessian block, a grid value outside the alphabet) reports picks 0, the all-zero payload and
+    // a NaN objective.
+    const bool tainted = grid_bad || h_bad || row_bad;
 
     // ---- the final objective Delta^T H Delta = sum_i cur_i grad_i: lane c sums columns
     // 16c .. 16c + 15 by a pairwise tree, then the butterfly joins the 16 lanes pairwise
     if (p.objective != nullptr && active) {
         float pr[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) pr[j] = __fmul_rn(cur[16 * c + j], grad[16 * c + j]);
+        for (int j = 0; j < 16; ++j) pr[j] = __fmul_rn(curT[(16 * c + j) * kRows + hr], grad[16 * c + j]);
         float t = tree_sum<16>(pr);
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1) t = __fadd_rn(t, __shfl_xor_sync(hmask, t, o));
-        if (c == 0) p.objective[row * p.nblk + blk] = t;
+        if (c == 0) p.objective[row * p.nblk + blk] = tainted ? __uint_as_float(0x7FC00000u) : t;
+    }
+
+    // ---- the final Delta (one block per launch): what the per-block calibration loop
+    // propagates; a row-block with a finding has the all-zero payload, so its Delta is x
+    if (p.delta_out != nullptr && active) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            float xv[8], dv[8];
+            load_x8<F32>(xrow, 2 * c + t, xv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dv[j] = tainted ? xv[j] : curT[(16 * c + 8 * t + j) * kRows + hr];
+            float4* dst = reinterpret_cast<float4*>(p.delta_out + row * kBlock + 16 * c + 8 * t);
+            dst[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+            dst[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+        }
     }
 
     // ---- step 4: picks and the payload assembled from the picked candidates
     if (active) {
         __syncwarp(hmask);
-        for (int q = c; q < G; q += 16) p.picks[(row * p.nblk + blk) * G + q] = static_cast<uint8_t>(C::PICK0 + pick[q]);
+        for (int q = c; q < G; q += 16)
+            p.picks[(row * p.nblk + blk) * G + q] = static_cast<uint8_t>(C::PICK0 + (tainted ? 0 : pick[q]));
     }
     if (!C::G8 && active) {  // 8-column groups report picks only: no payload stores their scales
         uint8_t* out = p.payload + (row * p.payload_ld + blk) * C::B;
@@ -568,18 +646,18 @@ __global__ void __launch_bounds__(Cfg<FMT>::T) choice_search_kernel(const Choice
                 const int g = i < 34 ? (i - 2) >> 2 : (i - 34) >> 1;
                 v = cand[pick[g] * C::B + i];
             }
-            out[i] = v;
+            out[i] = tainted ? static_cast<uint8_t>(0) : v;
         }
     }
 }
 
-template <int FMT>
+template <int FMT, bool F32>
 cudaError_t launch(const ChoiceParams& p, cudaStream_t s) {
     using C = Cfg<FMT>;
-    auto kern = choice_search_kernel<FMT>;
+    auto kern = choice_search_kernel<FMT, F32>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::smem);
     if (err != cudaSuccess) return err;
-    const int64_t ctas = p.nblk * (p.rows / p.rows_per_hess) * ((p.rows_per_hess + C::R - 1) / C::R);
+    const int64_t ctas = p.nblk_run * (p.rows / p.rows_per_hess) * ((p.rows_per_hess + C::R - 1) / C::R);
     kern<<<static_cast<unsigned>(ctas), C::T, C::smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -594,12 +672,19 @@ __global__ void sqrt_diag_kernel(const float* hess, int64_t nblk, float* out) {
 }  // namespace
 
 cudaError_t launch_choice_search(int fmt, const ChoiceParams& p, int /*num_sms*/, cudaStream_t s) {
-    if (p.rows == 0 || p.nblk == 0) return cudaSuccess;
-    if (fmt == IQ_FMT_IQ1_S) return launch<IQ_FMT_IQ1_S>(p, s);
-    if (fmt == IQ_FMT_IQ2_S) return launch<IQ_FMT_IQ2_S>(p, s);
-    if (fmt == IQ_FMT_IQ1_M) return launch<IQ_FMT_IQ1_M>(p, s);
-    if (fmt == kChoiceIq2xsG8) return launch<kChoiceIq2xsG8>(p, s);
-    return launch<IQ_FMT_IQ2_XS>(p, s);
+    if (p.rows == 0 || p.nblk_run == 0) return cudaSuccess;
+    if (p.w_f32) {  // the per-block calibration loop's compensated weights
+        if (fmt == IQ_FMT_IQ1_S) return launch<IQ_FMT_IQ1_S, true>(p, s);
+        if (fmt == IQ_FMT_IQ2_S) return launch<IQ_FMT_IQ2_S, true>(p, s);
+        if (fmt == IQ_FMT_IQ1_M) return launch<IQ_FMT_IQ1_M, true>(p, s);
+        if (fmt == IQ_FMT_IQ2_XS) return launch<IQ_FMT_IQ2_XS, true>(p, s);
+        return cudaErrorInvalidValue;
+    }
+    if (fmt == IQ_FMT_IQ1_S) return launch<IQ_FMT_IQ1_S, false>(p, s);
+    if (fmt == IQ_FMT_IQ2_S) return launch<IQ_FMT_IQ2_S, false>(p, s);
+    if (fmt == IQ_FMT_IQ1_M) return launch<IQ_FMT_IQ1_M, false>(p, s);
+    if (fmt == kChoiceIq2xsG8) return launch<kChoiceIq2xsG8, false>(p, s);
+    return launch<IQ_FMT_IQ2_XS, false>(p, s);
 }
 
 cudaError_t launch_sqrt_diag(const float* hess, int64_t nblk, float* out, cudaStream_t s) {

@@ -214,6 +214,10 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
  * its own H_gg; grad = H Delta; two sweeps over the groups in order, each taking the choice with
  * the least gain 2 u^T grad_g + u^T H_gg u (u = Delta_g(c) - Delta_g(cur)) iff that gain < 0,
  * then grad += H[:, g] u. Lowest choice on equal score or gain.
+ * Findings (IQ_FLAG_NONFINITE: a non-finite weight in the row-block or a non-finite entry of its
+ * Hessian block; IQ_FLAG_GRID: a grid value outside the candidates' alphabet) make that
+ * row-block report picks 0 (the first candidate), the all-zero payload and a NaN objective
+ * (bits 0x7FC00000); the other row-blocks are unaffected.
  */
 iq_status iq_choice_search(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t nblk,
                            int64_t ldw, const float *hess, int64_t rows_per_hess, const uint8_t *cand,
@@ -234,6 +238,36 @@ iq_status iq_choice_search_g8(const iq_desc *desc, const uint16_t *w, int64_t ro
                               const float *hess, int64_t rows_per_hess, const uint8_t *cand, int64_t cand_ld,
                               int64_t cand_choice_stride, uint8_t *picks, float *objective, uint32_t *flags,
                               cudaStream_t stream);
+
+/*
+ * The per-block calibration loop over one weight in a single call (PR #3218: "GPTQ with
+ * local_hessian_scales searches one block at a time"), with GPTQ's error propagation between the
+ * blocks (Frantar et al. 2022, "GPTQ: Accurate Post-Training Quantization for Generative
+ * Pre-trained Transformers", one 256-column block per lazy batch). Every row independently:
+ *   w_work = fp32(w); for b = 0 .. cols/256 - 1, in order:
+ *     x = w_work[:, block b]; the every-choice encode of x under importance sqrt(diag H_b);
+ *     the local-Hessian choice search of x under H_b (iq_choice_search's steps and findings)
+ *       -> picks[:, b], payload[:, b] and E = x - decode(payload[:, b]);
+ *     Y = E U_bb^-1 (forward substitution: column j starts from E_j, takes fma(-Y_k, U[k][j], .)
+ *       for k < j ascending, then Y_j = acc / U[j][j]); every later column j' of w_work takes
+ *       fma(-Y_k, U[256 b + k][j'], .) for k = 0..255 ascending.
+ *   U is the upper-triangular Cholesky factor of the weight's inverse Hessian (H^-1 = U^T U),
+ *   fp32 [cols][ldu], read on and above the diagonal; block b's local Hessian is
+ *   H_b = U_bb^-1 U_bb^-T, given in hess [cols/256][256][256] as iq_choice_search reads it.
+ *   w: bf16 [rows][ldw]; payload [rows][cols/256][B]; picks [rows][cols/256][G];
+ *   w_work: fp32 [rows][cols], caller-owned output: on return its block b holds the weights
+ *     block b was quantised from.
+ *   workspace: device scratch of at least iq_gptq_workspace_bytes(fmt, rows) bytes, 256-byte
+ *     aligned, owned by the caller (the candidates of one block, its error and its importance);
+ *     its contents on return mean nothing.
+ * All blocks are enqueued on `stream` in order, with no host synchronisation between them (with a
+ * flags word; without one the call waits at its end, as every call does). Alignment: w, hess, U
+ * and w_work 16-byte aligned, ldw a multiple of 8, ldu of 4 (IQ_EINVAL otherwise).
+ */
+size_t iq_gptq_workspace_bytes(int32_t fmt, int64_t rows);
+iq_status iq_gptq_blocks(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t cols, int64_t ldw,
+                         const float *hess, const float *U, int64_t ldu, void *workspace, size_t workspace_bytes,
+                         uint8_t *payload, uint8_t *picks, float *w_work, uint32_t *flags, cudaStream_t stream);
 
 /*
  * out[b * 256 + i] = sqrtf(hess[b][i][i]) for b < nblk: the search importance the local-Hessian
