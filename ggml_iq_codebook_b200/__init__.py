@@ -34,7 +34,8 @@ IQ_IN = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
 
 SYMBOLS = ("iq_block_bytes", "iq_payload_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
-           "iq_choice_search", "iq_choice_search_g8", "iq_gptq_workspace_bytes", "iq_gptq_blocks", "iq_sqrt_diag",
+           "iq_choice_search", "iq_choice_search_g8", "iq_gptq_workspace_bytes", "iq_gptq_blocks",
+           "iq_gptq_blocks_static", "iq_sqrt_diag",
            "iq_status_string", "iq_build_info")
 PROBE_SYMBOLS = ("iq_probe_fp32", "iq_probe_fp32_ops_per_iter")  # include/iq_probe.h: measurement only
 
@@ -83,6 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.iq_gptq_blocks.restype = ctypes.c_int
     lib.iq_gptq_blocks.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, P, i64, P, ctypes.c_size_t, P, P, P,
                                    P, P]
+    lib.iq_gptq_blocks_static.restype = ctypes.c_int
+    lib.iq_gptq_blocks_static.argtypes = [ctypes.POINTER(IQDesc), P, i64, i64, i64, P, P, i64, P, P, P, P, P]
     lib.iq_sqrt_diag.restype = ctypes.c_int
     lib.iq_sqrt_diag.argtypes = [P, i64, P, P]
     lib.iq_status_string.restype = ctypes.c_char_p

@@ -410,6 +410,7 @@ const char* iq_status_string(iq_status s) {
         case IQ_ERANGE: return "a block scale overflows fp16, or a given scale is negative, infinite or NaN";
         case IQ_ECHOICE: return "a given choice is out of the format's range";
         case IQ_EGRID: return "a grid value lies outside the format's alphabet";
+        case IQ_ESCRATCH: return "the call needs more scratch than the library's static 10 MiB array";
         default: return "unknown status";
     }
 }

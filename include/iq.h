@@ -68,7 +68,8 @@ typedef enum {
     IQ_EIMPORTANCE = 6,   /* an importance value is NaN, infinite or negative (PR #2723 review)  */
     IQ_ERANGE = 7,        /* d rounds to fp16 infinity, or a given d is negative, infinite or NaN */
     IQ_ECHOICE = 8,       /* a given choice is >= the format's number of choices              */
-    IQ_EGRID = 9          /* a grid value lies outside the format's alphabet                   */
+    IQ_EGRID = 9,         /* a grid value lies outside the format's alphabet                   */
+    IQ_ESCRATCH = 10      /* iq_gptq_blocks_static: the call needs more than the library's 10 MiB */
 } iq_status;
 
 typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3, IQ_FMT_IQ2_S = 4 } iq_format;
@@ -268,6 +269,27 @@ size_t iq_gptq_workspace_bytes(int32_t fmt, int64_t rows);
 iq_status iq_gptq_blocks(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t cols, int64_t ldw,
                          const float *hess, const float *U, int64_t ldu, void *workspace, size_t workspace_bytes,
                          uint8_t *payload, uint8_t *picks, float *w_work, uint32_t *flags, cudaStream_t stream);
+
+/*
+ * iq_gptq_blocks without a workspace argument, for callers that cannot allocate device memory
+ * where they call it: code inside another framework's memory pool, which owns the free HBM;
+ * code held to a fixed device-memory budget from the moment it was loaded; code on a path where
+ * cudaMalloc's implicit device synchronisation cannot be afforded. The pages have no counterpart:
+ * this entry point exists for those callers only.
+ *   Scratch: a 10 MiB device array inside the library (every GPU that loads the library holds one
+ *   until the process exits). Calls whose iq_gptq_workspace_bytes(fmt, rows) exceeds 10 MiB get
+ *   IQ_ESCRATCH and enqueue nothing; 10 MiB covers 4096 rows in every format.
+ *   Set-up: the first call on a device looks up that device's address of the array (with the
+ *   device current); make that first call before any stream capture.
+ *   Sharing: every call uses the same array and leaves its contents behind. Nothing in it needs
+ *   clearing (each call writes every scratch byte it reads), but calls that overlap on the GPU,
+ *   from two streams or two host threads, race on it: order them.
+ *   Everything else (arguments, outputs, findings, statuses) is exactly iq_gptq_blocks's, and
+ *   the call allocates no device memory.
+ */
+iq_status iq_gptq_blocks_static(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t cols, int64_t ldw,
+                                const float *hess, const float *U, int64_t ldu, uint8_t *payload, uint8_t *picks,
+                                float *w_work, uint32_t *flags, cudaStream_t stream);
 
 /*
  * out[b * 256 + i] = sqrtf(hess[b][i][i]) for b < nblk: the search importance the local-Hessian
