@@ -199,17 +199,16 @@ __device__ __forceinline__ float tree_sum(float p[N]) {
     return p[0];
 }
 
-// Argmin over the 16 lanes of a half-warp of (key(value), choice): lowest choice on ties.
-__device__ __forceinline__ void half_argmin(float v, int c, unsigned mask, float& best, int& cbest) {
-    float k = argmin_key(v);
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) {
-        const float ko = __shfl_xor_sync(mask, k, o);
-        const int co = __shfl_xor_sync(mask, c, o);
-        if (ko < k || (ko == k && co < c)) { k = ko; c = co; }
-    }
-    best = k;
-    cbest = c;
+// Argmin over the 16 lanes of a half-warp of (key(value), choice), lowest choice on ties, where
+// lane c of the half-warp holds choice c. The key (NaN and +inf as +inf, -0 as +0, so that equal
+// floats are equal keys) is mapped to an order-preserving unsigned and reduced with one redux;
+// the lowest lane holding the minimum is the choice.
+__device__ __forceinline__ void half_argmin(float v, int /*c*/, unsigned mask, float& best, int& cbest) {
+    const uint32_t u = __float_as_uint(__fadd_rn(argmin_key(v), 0.0f));
+    const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t m = __reduce_min_sync(mask, o);
+    cbest = (__ffs(__ballot_sync(mask, o == m) & mask) - 1) & 15;
+    best = __uint_as_float((m & 0x80000000u) ? (m & 0x7FFFFFFFu) : ~m);
 }
 
 // v[i] = sum over k < W (fma chain, k ascending, starting from the product) of

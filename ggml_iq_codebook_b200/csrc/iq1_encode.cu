@@ -75,6 +75,28 @@ __device__ __forceinline__ Terms entry_terms(const char* smem, uint32_t lane_bas
     return t;
 }
 
+// The same terms with both shifts side by side, A = (A_+, A_-) and C = (C_+, C_-), so that one
+// packed fma.rn.f32x2 scores an entry under both shifts of a local scale. Every element is the
+// scalar version's op sequence (the packed ops are independent IEEE operations per element).
+struct Terms2 {
+    float2 A, C;
+};
+
+__device__ __forceinline__ Terms2 entry_terms2(const char* smem, uint32_t lane_base, uint4 o, float2 W2,
+                                               float Tall) {
+    const float2 plo = *reinterpret_cast<const float2*>(smem + lane_base + o.x);
+    const float2 phi = *reinterpret_cast<const float2*>(smem + lane_base + o.y);
+    const float2 nlo = *reinterpret_cast<const float2*>(smem + lane_base + o.z);
+    const float2 nhi = *reinterpret_cast<const float2*>(smem + lane_base + o.w);
+    const float2 p = __fadd2_rn(plo, phi), n = __fadd2_rn(nlo, nhi);  // (Wp, Tp), (Wn, Tn)
+    const float A = __fadd_rn(p.x, n.x), R = __fsub_rn(p.x, n.x), C = __fsub_rn(p.y, n.y);
+    Terms2 t;
+    t.A = __ffma2_rn(make_float2(0.015625f, 0.015625f), W2,
+                     make_float2(__fmaf_rn(0.25f, R, A), __fmaf_rn(-0.25f, R, A)));
+    t.C = make_float2(__fmaf_rn(0.125f, Tall, C), __fmaf_rn(-0.125f, Tall, C));
+    return t;
+}
+
 template <int BYTES>
 __device__ __forceinline__ void write_zero_block(uint8_t* out, int lane) {
     for (int i = lane; i < BYTES / 2; i += 32) reinterpret_cast<uint16_t*>(out)[i] = 0;
@@ -269,25 +291,32 @@ __global__ void __launch_bounds__(kWarps * 32, 2) iq1_encode_kernel(const Encode
             int bch[kChoices];
 #pragma unroll
             for (int c = 0; c < kChoices; ++c) { best[c] = INFINITY; bch[c] = 0; }
+            // m for both shifts of a local scale in one packed fma: (s, s) * (A_+, A_-) + (C_+, C_-)
+            const float2 W2 = make_float2(W, W);
+            float2 s2[8];
+#pragma unroll
+            for (int ls = 0; ls < 8; ++ls) s2[ls] = make_float2(s[ls], s[ls]);
             for (int ch = 0; ch < kIq1sEntries / K; ++ch) {
                 float cm[kChoices];
                 {
-                    const Terms ta = entry_terms(smem, lane_base, sgrid[ch * K], W, Tall);
-                    const Terms tb = entry_terms(smem, lane_base, sgrid[ch * K + 1], W, Tall);
+                    const Terms2 ta = entry_terms2(smem, lane_base, sgrid[ch * K], W2, Tall);
+                    const Terms2 tb = entry_terms2(smem, lane_base, sgrid[ch * K + 1], W2, Tall);
 #pragma unroll
                     for (int ls = 0; ls < 8; ++ls) {
-                        cm[ls] = fminf(__fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
-                        cm[8 + ls] = fminf(__fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
+                        const float2 ma = __ffma2_rn(s2[ls], ta.A, ta.C), mb = __ffma2_rn(s2[ls], tb.A, tb.C);
+                        cm[ls] = fminf(ma.x, mb.x);
+                        cm[8 + ls] = fminf(ma.y, mb.y);
                     }
                 }
 #pragma unroll 2
                 for (int q = ch * K + 2; q < ch * K + K; q += 2) {
-                    const Terms ta = entry_terms(smem, lane_base, sgrid[q], W, Tall);
-                    const Terms tb = entry_terms(smem, lane_base, sgrid[q + 1], W, Tall);
+                    const Terms2 ta = entry_terms2(smem, lane_base, sgrid[q], W2, Tall);
+                    const Terms2 tb = entry_terms2(smem, lane_base, sgrid[q + 1], W2, Tall);
 #pragma unroll
                     for (int ls = 0; ls < 8; ++ls) {
-                        cm[ls] = min3f(cm[ls], __fmaf_rn(s[ls], ta.Ap, ta.Cp), __fmaf_rn(s[ls], tb.Ap, tb.Cp));
-                        cm[8 + ls] = min3f(cm[8 + ls], __fmaf_rn(s[ls], ta.An, ta.Cn), __fmaf_rn(s[ls], tb.An, tb.Cn));
+                        const float2 ma = __ffma2_rn(s2[ls], ta.A, ta.C), mb = __ffma2_rn(s2[ls], tb.A, tb.C);
+                        cm[ls] = min3f(cm[ls], ma.x, mb.x);
+                        cm[8 + ls] = min3f(cm[8 + ls], ma.y, mb.y);
                     }
                 }
 #pragma unroll

@@ -34,9 +34,10 @@ constexpr int kMinCtas = 1;      // launch-bounds occupancy hint (CTAs per SM)
 constexpr int kTileBlocks = 256;  // blocks per staged payload tile
 constexpr int kCtasPerSm = 5;     // persistent CTAs per SM
 
+// Two fp32 values rounded to bf16 (nearest even) in one packed conversion: a in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void st_global_v8(void* ptr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
