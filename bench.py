@@ -229,6 +229,10 @@ WORKLOADS = {
                                          + ", the search as one call per 256-column block (16 calls)"),
     "iq1s_decode_1m_blocks": ("iq1_s", [4096, 4096], "IQ1_S bf16 decode of 1,048,576 blocks (the 4096x4096 "
                               "weighted payload x16)"),
+    "iq2xs_decode_1m_blocks": ("iq2_xs", [8192, 4096], "IQ2_XS bf16 decode of 1,048,576 blocks (the 8192x4096 "
+                               "payload x8)"),
+    "iq1m_decode_1m_blocks": ("iq1_m", [4096, 4096], "IQ1_M bf16 decode of 1,048,576 blocks (the 4096x4096 "
+                              "weighted payload x16)"),
     "gptq_iq2xs_4096x4096": ("iq2_xs", [4096, 4096], "per-block calibration loop in one call: for each 256-column "
                              "block in order, sqrt(diag H_b) + IQ2_XS every-choice encode + two-sweep local-Hessian "
                              "search + GPTQ propagation of its error to the later columns; 4096x4096 bf16 "
@@ -275,10 +279,13 @@ class Workload:
                 self.launches_per_step = 2 + self.w.shape[-1] // 256
         elif name.startswith("gptq_"):
             self._gptq(synth.workload_gptq_iq2xs(), text)
-        elif name == "iq1s_decode_1m_blocks":
-            self._encode_decode(synth.workload_iq1s_4096x4096_weighted(), text)
+        elif name.endswith("_decode_1m_blocks"):
+            base = {"iq1s": synth.workload_iq1s_4096x4096_weighted(), "iq1m": dict(
+                synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m"), "iq2xs": synth.workload_iq2xs_8192x4096()}
+            self._encode_decode(base[name.split("_")[0]], text)
             self.kind = "decode"
-            self.payload = self.payload.reshape(-1, 50).repeat(16, 1)
+            B = iq.BLOCK_BYTES[self.fmt]
+            self.payload = self.payload.reshape(-1, B).repeat((1 << 20) // (self.payload.numel() // B), 1)
             self.decoded = torch.empty((self.payload.shape[0], 256), dtype=torch.bfloat16, device=self.dev)
             self.units = self.payload.shape[0] * 256
             self.nblocks = self.payload.shape[0]
@@ -500,8 +507,9 @@ def decode_roofline(wl: Workload, dev, peaks):
     nbytes = nblocks * (B + 512)
     gbs = nbytes / ms / 1e6
     del big, out, flush
-    if wl.fmt == "iq1_s":
-        traffic, note = kernel_traffic("decode_kernel", "iq1s_decode_1m_blocks", nblocks)
+    name = {"iq1_s": "iq1s_decode_1m_blocks", "iq2_xs": "iq2xs_decode_1m_blocks", "iq1_m": "iq1m_decode_1m_blocks"}
+    if wl.fmt in name:
+        traffic, note = kernel_traffic("decode_kernel", name[wl.fmt], nblocks)
     else:
         traffic, note = None, f"no capture of the {wl.fmt} decode"
     return {"kernel": "decode_kernel (bf16 out)", "blocks": nblocks, "bytes_per_launch": nbytes,
@@ -552,6 +560,8 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
             wl = {"iq1s_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
                   "iq1m_4096x4096_weighted": synth.workload_iq1s_4096x4096_weighted,
                   "iq1s_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
+                  "iq1m_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
+                  "iq2xs_decode_1m_blocks": synth.workload_iq2xs_8192x4096,
                   "iq2xs_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq2s_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq1s_64x256": synth.workload_iq1s_64x256}[name]()

@@ -175,7 +175,7 @@ struct Cfg {
     static constexpr int oUT = oCurT + kBlock * R * 4;        // float [W][R]: u of the rows that switched
     static constexpr int oUR = oUT + W * R * 4;               // float [R][W]: the same, by row
     static constexpr int oT2 = oUR + R * W * 4;               // float [R][G][NC]: u^T H_gg u per candidate
-    static constexpr int oSw = oT2 + R * G * NC * 4;          // int [R]: row switched this step
+    static constexpr int oSw = oT2 + R * G * NC * 4;          // uint32 [2]: rows that switched, by step parity
     // update by column up to this many switched rows, else by tiles (either is bit-exact)
     static constexpr int COLUMN_MAX = W == 32 ? kColumnMaxW32 : kColumnMaxW16;
     static constexpr int oGrid = oSw + R * 4;                     // uint16 [E] element codes
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     float* curT = reinterpret_cast<float*>(smem + C::oCurT);
     float* uT = reinterpret_cast<float*>(smem + C::oUT);
     float* uR = reinterpret_cast<float*>(smem + C::oUR);
-    int* swf = reinterpret_cast<int*>(smem + C::oSw);
+    uint32_t* swbits = reinterpret_cast<uint32_t*>(smem + C::oSw);
     uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem + C::oGrid);
 
     // CTA -> (block, expert, row tile): a tile never straddles two experts, and the CTAs that
@@ -465,6 +465,22 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     h_bad = __syncthreads_or(h_bad);
     if (tid == 0) raise_flags(p.flags, (grid_bad ? IQ_FLAG_GRID : 0u) | (h_bad ? IQ_FLAG_NONFINITE : 0u));
     if (active && c == 0 && row_bad) raise_flags(p.flags, IQ_FLAG_NONFINITE);
+    // The gradient tiles wanted the rows' Delta by column; the sweeps read and write whole
+    // groups of one row, so the same area is rewritten row-major: cur[r][i].
+    float* cur = curT;
+    {
+        float v[kBlock * kRows / kThreads];
+#pragma unroll
+        for (int t = 0; t < kBlock * kRows / kThreads; ++t) v[t] = curT[tid + t * kThreads];
+        __syncthreads();
+#pragma unroll
+        for (int t = 0; t < kBlock * kRows / kThreads; ++t) {
+            const int idx = tid + t * kThreads;  // = i * kRows + r
+            cur[(idx % kRows) * kBlock + idx / kRows] = v[t];
+        }
+        if (tid == 0) swbits[0] = swbits[1] = 0u;
+    }
+    float* cur_row = cur + hr * kBlock;
 
     // ---- step 3: two sweeps over the groups. Each row decides (lane per choice) from the stored
     // curvature term and the current gradient; a row that switches in the first sweep rescores
@@ -481,7 +497,12 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
             float dl[W], u[W];
             delta_of(g, dl);
 #pragma unroll
-            for (int i = 0; i < W; ++i) u[i] = __fsub_rn(dl[i], curT[(g * W + i) * kRows + hr]);
+            {
+                float cg[W];
+                load_vec<W>(cur_row + g * W, cg);
+#pragma unroll
+                for (int i = 0; i < W; ++i) u[i] = __fsub_rn(dl[i], cg[i]);
+            }
             float gain;
             {
                 float gq[WO], p1[WO], up[WO];
@@ -504,7 +525,8 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
                     for (int i = 0; i < W; i += 4)
                         *reinterpret_cast<float4*>(uR + hr * W + i) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
 #pragma unroll
-                    for (int i = 0; i < W; ++i) curT[(g * W + i) * kRows + hr] = dl[i];
+                    for (int i = 0; i < W; i += 4)
+                        *reinterpret_cast<float4*>(cur_row + g * W + i) = make_float4(dl[i], dl[i + 1], dl[i + 2], dl[i + 3]);
                     pick[g] = c;
                 }
                 if (step < 2 * G) {  // the second sweep's curvature terms around the new pick
@@ -515,15 +537,14 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
                 }
             }
         }
-        if (c == 0) swf[hr] = switched;
+        if (c == 0 && switched) atomicOr(&swbits[step & 1], 1u << hr);
         __syncthreads();
         // grad[r][i] += sum_k H[k][i] u_k (fma chain over the group's k, the same order either
         // way) for the rows that switched. Few switches: by column, each thread holding H[k][i]
         // for its columns in registers and walking only those rows. Many: 4-row x 4-column
         // register tiles over every 4-row group with a switch, writing back only switched rows.
-        uint32_t swmask = 0;
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) swmask |= static_cast<uint32_t>(swf[r] != 0) << r;
+        const uint32_t swmask = swbits[step & 1];
+        if (tid == 0) swbits[(step + 1) & 1] = 0u;  // every thread read it last step, before this step's first barrier
         if (swmask != 0 && __popc(swmask) <= C::COLUMN_MAX) {
 #pragma unroll
             for (int i = tid; i < kBlock; i += kThreads) {
@@ -574,7 +595,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     if (p.objective != nullptr && active) {
         float pr[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) pr[j] = __fmul_rn(curT[(16 * c + j) * kRows + hr], grad[16 * c + j]);
+        for (int j = 0; j < 16; ++j) pr[j] = __fmul_rn(cur_row[16 * c + j], grad[16 * c + j]);
         float t = tree_sum<16>(pr);
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1) t = __fadd_rn(t, __shfl_xor_sync(hmask, t, o));
@@ -589,7 +610,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
             float xv[8], dv[8];
             load_x8<F32>(xrow, 2 * c + t, xv);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) dv[j] = tainted ? xv[j] : curT[(16 * c + 8 * t + j) * kRows + hr];
+            for (int j = 0; j < 8; ++j) dv[j] = tainted ? xv[j] : cur_row[16 * c + 8 * t + j];
             float4* dst = reinterpret_cast<float4*>(p.delta_out + row * kBlock + 16 * c + 8 * t);
             dst[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
             dst[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);

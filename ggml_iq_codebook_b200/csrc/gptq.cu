@@ -10,8 +10,9 @@
 //       for k < j ascending, and Y_j = acc / U[j][j] (IEEE division);
 //   every later column j' starts from w[j'] and takes fma(-Y_k, U[b 256 + k][j'], .) for
 //       k = 0..255 ascending.
-// Design (B200): the solve runs a warp per row, lane L owning columns 8L..8L+7 (each Y_k is
-// broadcast by one shuffle and all later columns advance their chains at once); the update is an
+// Design (B200): the solve runs a warp per row, lane L owning columns 8L..8L+7 (a lane resolves
+// its 8 columns, one shuffle round broadcasts them, all later columns advance their chains; the
+// CTA's rows share U_bb's rows through shared memory); the update is an
 // FP32 register-tiled GEMM (8 rows x 8 columns per thread, k staged through shared memory in
 // ascending chunks) whose column pairs run as packed fma.rn.f32x2, so every output is still one
 // sequential IEEE fma chain over k.
@@ -36,39 +37,78 @@ __global__ void bf16_to_f32_kernel(const uint16_t* w, int64_t rows, int64_t cols
 
 constexpr int kSolveWarps = 8;
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // e [rows][256] holds E on entry and Y = E U_bb^-1 on exit; ubb points at U[o][o], row stride ldu.
+// A warp per row, lane L owning columns 8L..8L+7. Column group kb resolves in one lane: lane kb
+// takes its 8 Y's in order (each division, then the fmas into its own later columns), broadcasts
+// them, and every later lane applies the 8 to its columns, k ascending -- the forward
+// substitution's chains in the oracle's order, with one cross-lane round trip per 8 columns.
+// The CTA's warps share the rows 8 kb .. 8 kb + 7 of U_bb, staged in shared memory (double
+// buffered with cp.async: the next group's 8 KiB stream in while this group resolves). A row's
+// 16-byte slots are stored swizzled (slot q at q ^ (q >> 3 & 1)) so that a warp's reads of its
+// lanes' 32-byte column chunks spread over every bank.
 __global__ void __launch_bounds__(32 * kSolveWarps) gptq_solve_kernel(float* e, const float* ubb, int64_t ldu,
                                                                       int64_t rows) {
+    __shared__ __align__(16) float us[2][8][kBlock];
+    auto swz = [](int q) { return q ^ ((q >> 3) & 1); };  // 16-byte slot of logical slot q
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kSolveWarps + (threadIdx.x >> 5);
-    if (row >= rows) return;  // warp-uniform
-    float* er = e + row * kBlock + 8 * lane;
-    float acc[8], y[8];
-    {
+    const bool active = row < rows;
+    auto stage = [&](int kb, int buf) {
+        for (int i = threadIdx.x; i < 8 * kBlock / 4; i += 32 * kSolveWarps) {
+            const int r = i / (kBlock / 4), c4 = i - r * (kBlock / 4);
+            cp_async16(&us[buf][r][4 * swz(c4)], ubb + (8 * kb + r) * ldu + 4 * c4);
+        }
+        cp_async_commit();
+    };
+    float* er = e + (active ? row : 0) * kBlock + 8 * lane;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0}, y[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (active) {
         const float4 a = reinterpret_cast<const float4*>(er)[0], b = reinterpret_cast<const float4*>(er)[1];
         acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w; acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
     }
+    stage(0, 0);
 #pragma unroll 1
     for (int kb = 0; kb < 32; ++kb) {
+        cp_async_wait_all();
+        __syncthreads();  // group kb's rows have landed; every warp is done with the other buffer
+        if (kb + 1 < 32) stage(kb + 1, (kb + 1) & 1);
+        const float(*u)[kBlock] = us[kb & 1];
+        auto at = [&](int r, int c) { return u[r][4 * swz(c >> 2) + (c & 3)]; };  // U[8 kb + r][c]
+        float ys[8];
+        if (lane == kb) {
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const int k = 8 * kb + s;
-            const float* uk = ubb + k * ldu + 8 * lane;  // U[k][8 lane .. 8 lane + 7]
-            const float4 u0 = __ldg(reinterpret_cast<const float4*>(uk)), u1 = __ldg(reinterpret_cast<const float4*>(uk) + 1);
-            float yk = 0.0f;
-            if (lane == kb) {
-                yk = __fdiv_rn(acc[s], __ldg(ubb + k * ldu + k));
-                y[s] = yk;
+            for (int s = 0; s < 8; ++s) {
+                ys[s] = __fdiv_rn(acc[s], at(s, 8 * kb + s));  // U[k][k], k = 8 kb + s
+                y[s] = ys[s];
+#pragma unroll
+                for (int t = s + 1; t < 8; ++t) acc[t] = __fmaf_rn(-ys[s], at(s, 8 * kb + t), acc[t]);
             }
-            yk = __shfl_sync(0xffffffffu, yk, kb);
-            const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        }
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (8 * lane + i > k) acc[i] = __fmaf_rn(-yk, uv[i], acc[i]);
+        for (int s = 0; s < 8; ++s) ys[s] = __shfl_sync(0xffffffffu, ys[s], kb);
+        if (lane > kb) {
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const float4 ua = *reinterpret_cast<const float4*>(&u[s][4 * swz(2 * lane)]);
+                const float4 ub = *reinterpret_cast<const float4*>(&u[s][4 * swz(2 * lane + 1)]);
+                const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(-ys[s], uv[i], acc[i]);
+            }
         }
     }
-    reinterpret_cast<float4*>(er)[0] = make_float4(y[0], y[1], y[2], y[3]);
-    reinterpret_cast<float4*>(er)[1] = make_float4(y[4], y[5], y[6], y[7]);
+    cp_async_wait_all();
+    if (active) {
+        reinterpret_cast<float4*>(er)[0] = make_float4(y[0], y[1], y[2], y[3]);
+        reinterpret_cast<float4*>(er)[1] = make_float4(y[4], y[5], y[6], y[7]);
+    }
 }
 
 constexpr int kBM = 128, kBN = 128, kBK = 16, kUpdThreads = 256;
