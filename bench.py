@@ -233,6 +233,8 @@ WORKLOADS = {
                                "payload x8)"),
     "iq1m_decode_1m_blocks": ("iq1_m", [4096, 4096], "IQ1_M bf16 decode of 1,048,576 blocks (the 4096x4096 "
                               "weighted payload x16)"),
+    "iq2s_decode_1m_blocks": ("iq2_s", [8192, 4096], "IQ2_S bf16 decode of 1,048,576 blocks (the 8192x4096 "
+                              "payload x8)"),
     "gptq_iq2xs_4096x4096": ("iq2_xs", [4096, 4096], "per-block calibration loop in one call: for each 256-column "
                              "block in order, sqrt(diag H_b) + IQ2_XS every-choice encode + two-sweep local-Hessian "
                              "search + GPTQ propagation of its error to the later columns; 4096x4096 bf16 "
@@ -281,7 +283,8 @@ class Workload:
             self._gptq(synth.workload_gptq_iq2xs(), text)
         elif name.endswith("_decode_1m_blocks"):
             base = {"iq1s": synth.workload_iq1s_4096x4096_weighted(), "iq1m": dict(
-                synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m"), "iq2xs": synth.workload_iq2xs_8192x4096()}
+                synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m"), "iq2xs": synth.workload_iq2xs_8192x4096(),
+                "iq2s": dict(synth.workload_iq2xs_8192x4096(), fmt="iq2_s")}
             self._encode_decode(base[name.split("_")[0]], text)
             self.kind = "decode"
             B = iq.BLOCK_BYTES[self.fmt]
@@ -507,7 +510,8 @@ def decode_roofline(wl: Workload, dev, peaks):
     nbytes = nblocks * (B + 512)
     gbs = nbytes / ms / 1e6
     del big, out, flush
-    name = {"iq1_s": "iq1s_decode_1m_blocks", "iq2_xs": "iq2xs_decode_1m_blocks", "iq1_m": "iq1m_decode_1m_blocks"}
+    name = {"iq1_s": "iq1s_decode_1m_blocks", "iq2_xs": "iq2xs_decode_1m_blocks", "iq1_m": "iq1m_decode_1m_blocks",
+            "iq2_s": "iq2s_decode_1m_blocks"}
     if wl.fmt in name:
         traffic, note = kernel_traffic("decode_kernel", name[wl.fmt], nblocks)
     else:
@@ -562,6 +566,7 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
                   "iq1s_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
                   "iq1m_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
                   "iq2xs_decode_1m_blocks": synth.workload_iq2xs_8192x4096,
+                  "iq2s_decode_1m_blocks": synth.workload_iq2xs_8192x4096,
                   "iq2xs_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq2s_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq1s_64x256": synth.workload_iq1s_64x256}[name]()
@@ -740,7 +745,8 @@ def main():
         cpu = {"value": round(rate, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"first {rows} rows x {cols} cols of the workload, encode + decode, {dt:.1f} s wall"}
 
-    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    metric = "IQ decode Mweights/s" if wl.kind == "decode" else METRIC
+    line = {"metric": metric, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
             "roofline": roof, "decode": dec, "cpu_baseline": cpu,
