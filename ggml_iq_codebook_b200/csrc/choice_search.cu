@@ -35,9 +35,13 @@
 // done by all threads together: the initial H Delta as 4-row x 4-column register tiles (per k one
 // 16-byte read of the rows' values and one of H, then 16 fmas); after a sweep step, by column when
 // few rows switched (each thread holding its H column and walking only those rows), else by the
-// same tiles. The grid is staged as 16-bit element codes, so decoding needs no int-to-float
-// conversions. On request each row's final Delta^T H Delta is reported as sum_i cur_i grad_i (a
-// pairwise tree over the 256 columns).
+// same tiles. The grid is staged per format so that decoding needs no int-to-float conversion:
+// IQ1 as 16-bit +1/-1 masks, each element selecting among its group's three values; IQ2 as
+// byte-permute selectors over tables of the four magnitudes' 16-bit halves (two permutes per
+// pair of halves, two to join them into floats, the signs by XOR). The block's H is checked for
+// non-finite entries through the initial gradient: every entry enters a chain of every row, so
+// the explicit scan runs only in a CTA whose gradient came out non-finite. On request each row's
+// final Delta^T H Delta is reported as sum_i cur_i grad_i (a pairwise tree over the 256 columns).
 #include "iq_device.cuh"
 #include "iq_kernels.h"
 
@@ -53,28 +57,59 @@ __device__ __forceinline__ void load_vec(const float* src, float v[N]) {
     }
 }
 
-// The grid staged as 16-bit element codes: IQ1_S and IQ1_M (+1 mask) | (-1 mask) << 8; IQ2_XS and
-// IQ2_S two bits (g - 1) / 2 per element.
-template <int FMT>
-__device__ __forceinline__ uint16_t grid_code(int2 raw) {
+// An IQ1 grid entry as masks: bit j set when q_j = +1, bit 8 + j when q_j = -1.
+__device__ __forceinline__ uint16_t grid_masks(int2 raw) {
     uint32_t c = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
-        if (FMT == IQ_FMT_IQ1_S || FMT == IQ_FMT_IQ1_M)
-            c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
-        else
-            c |= (static_cast<uint32_t>((v - 1) >> 1) & 3u) << (2 * j);
+        c |= (static_cast<uint32_t>(v == 1) << j) | (static_cast<uint32_t>(v == -1) << (8 + j));
     }
     return static_cast<uint16_t>(c);
+}
+
+// An IQ2 grid entry as four byte-permute selectors, one per element pair (2p, 2p + 1) at bits
+// 16p..16p+15 of the 64-bit entry: nibbles (2 c0, 2 c0 + 1, 2 c1, 2 c1 + 1) pick the 16-bit
+// entries c0 and c1 of a four-entry table, c = (g - 1) / 2.
+__device__ __forceinline__ uint2 grid_selectors(int2 raw) {
+    uint32_t sel[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int v = static_cast<int8_t>(((j < 4 ? raw.x : raw.y) >> (8 * (j & 3))) & 0xFF);
+        const uint32_t c = static_cast<uint32_t>((v - 1) >> 1) & 3u;
+        sel[j >> 2] |= ((2u * c) | ((2u * c + 1u) << 4)) << (8 * (j & 3));
+    }
+    return make_uint2(sel[0], sel[1]);
+}
+
+// The 8 values m(c_j), negated where bit j of neg is set, with the four magnitudes (m1, m3, m5,
+// m7) split into a table of their low halves and one of their high halves: a pair's two low
+// halves are one byte permute, its two high halves another, and two more join them into the
+// pair's floats. The sign is the float's top bit, so negation is an XOR (also for zero).
+__device__ __forceinline__ void pick8(uint2 sel, float m1, float m3, float m5, float m7, uint32_t neg, float xh[8]) {
+    const uint32_t u1 = __float_as_uint(m1), u3 = __float_as_uint(m3), u5 = __float_as_uint(m5), u7 = __float_as_uint(m7);
+    const uint32_t la = __byte_perm(u1, u3, 0x5410), lb = __byte_perm(u5, u7, 0x5410);
+    const uint32_t ha = __byte_perm(u1, u3, 0x7632), hb = __byte_perm(u5, u7, 0x7632);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t w = p < 2 ? sel.x : sel.y;
+        const uint32_t sp = (p & 1) ? (w >> 16) : w;
+        const uint32_t lo = __byte_perm(la, lb, sp), hi = __byte_perm(ha, hb, sp);
+        const uint32_t e0 = __byte_perm(lo, hi, 0x5410) ^ ((neg << (31 - 2 * p)) & 0x80000000u);
+        const uint32_t e1 = __byte_perm(lo, hi, 0x7632) ^ ((neg << (30 - 2 * p)) & 0x80000000u);
+        xh[2 * p] = __uint_as_float(e0);
+        xh[2 * p + 1] = __uint_as_float(e1);
+    }
 }
 
 // The decoded values of one 8-weight group of candidate `pc`: xh[j] = value of element j of
 // 8-weight group `grp8` (inside the block) in choice group g. The products the group can take are
 // formed once (IQ1_S: s (q + delta), q in {-1, 0, 1}; IQ2_XS: s g, g in {1, 3, 5, 7}), each
-// rounded exactly as the direct formula rounds it, and picked per element (no int-to-float).
+// rounded exactly as the direct formula rounds it, and picked per element (no int-to-float) from
+// the staged grid: `sgrid_v` holds 16-bit masks for IQ1_S and IQ1_M, 64-bit selectors for IQ2.
 template <int FMT>
-__device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid, int g, int grp8, float xh[8]) {
+__device__ __forceinline__ void decode8(const uint8_t* pc, const void* sgrid_v, int g, int grp8, float xh[8]) {
+    const uint16_t* sgrid = static_cast<const uint16_t*>(sgrid_v);
     if (FMT == IQ_FMT_IQ1_M) {
         // 56-byte layout: low index byte grp8; its nibble in byte 32 + grp8 / 2 (3 high index
         // bits, bit 3 = delta -1/8); choice group g's 3-bit scale in word 48 + 2 (g / 4); d in
@@ -102,13 +137,7 @@ __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid
         const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
         const uint32_t idx = static_cast<uint32_t>(pc[2 + grp8]) | (((static_cast<uint32_t>(pc[66 + (grp8 >> 2)]) >> (2 * (grp8 & 3))) & 3u) << 8);
         const uint32_t neg = pc[34 + grp8];
-        const uint32_t e = sgrid[idx];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t cj = (e >> (2 * j)) & 3u;
-            const float a = (cj & 2u) ? ((cj & 1u) ? m7 : m5) : ((cj & 1u) ? m3 : m1);
-            xh[j] = ((neg >> j) & 1u) ? -a : a;
-        }
+        pick8(static_cast<const uint2*>(sgrid_v)[idx], m1, m3, m5, m7, neg, xh);
     } else if (FMT == IQ_FMT_IQ2_XS) {
         const uint32_t code = *reinterpret_cast<const uint16_t*>(pc + 2 + 2 * grp8);
         const uint32_t sc = pc[66 + (g >> 1)];
@@ -117,13 +146,7 @@ __device__ __forceinline__ void decode8(const uint8_t* pc, const uint16_t* sgrid
         const float m1 = __fmul_rn(s, 1.0f), m3 = __fmul_rn(s, 3.0f), m5 = __fmul_rn(s, 5.0f), m7 = __fmul_rn(s, 7.0f);
         const uint32_t sign7 = code >> 9;
         const uint32_t neg = sign7 | (static_cast<uint32_t>(__popc(sign7) & 1) << 7);
-        const uint32_t e = sgrid[code & 511u];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t cj = (e >> (2 * j)) & 3u;
-            const float a = (cj & 2u) ? ((cj & 1u) ? m7 : m5) : ((cj & 1u) ? m3 : m1);
-            xh[j] = ((neg >> j) & 1u) ? -a : a;
-        }
+        pick8(static_cast<const uint2*>(sgrid_v)[code & 511u], m1, m3, m5, m7, neg, xh);
     } else {
         const uint32_t qh = *reinterpret_cast<const uint16_t*>(pc + 34 + 2 * g);
         const float s = __fmul_rn(d, small_int_to_float(2u * ((qh >> 12) & 7u) + 1u));
@@ -178,8 +201,9 @@ struct Cfg {
     static constexpr int oSw = oT2 + R * G * NC * 4;          // uint32 [2]: rows that switched, by step parity
     // update by column up to this many switched rows, else by tiles (either is bit-exact)
     static constexpr int COLUMN_MAX = W == 32 ? kColumnMaxW32 : kColumnMaxW16;
-    static constexpr int oGrid = oSw + R * 4;                     // uint16 [E] element codes
-    static constexpr int oRows = oGrid + (E * 2 + 15) / 16 * 16;  // per-row records
+    static constexpr bool IQ2 = DF == IQ_FMT_IQ2_XS || DF == IQ_FMT_IQ2_S;
+    static constexpr int oGrid = oSw + R * 4;  // IQ2: uint2 [E] selectors; IQ1: uint16 [E] masks
+    static constexpr int oRows = oGrid + (IQ2 ? E * 8 : (E * 2 + 15) / 16 * 16);  // per-row records
     static constexpr int rGrad = 0;                               // float [256]
     static constexpr int rPick = rGrad + kBlock * 4;              // int [G]
     static constexpr int rCand = (rPick + G * 4 + 15) / 16 * 16;  // uint8 [16][B]
@@ -357,12 +381,13 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     };
     prefetch(0);
 
-    // ---- stage the grid codes (checking the alphabet) and the row's candidate payloads (lanes
+    // ---- stage the grid (checking the alphabet) and the row's candidate payloads (lanes
     // past the format's NC candidates stage zeros and never win); a non-finite weight taints the row
     bool grid_bad = false, h_bad = false, row_bad = false;
     for (int q = tid; q < C::E; q += kThreads) {
         const int2 raw = __ldg(reinterpret_cast<const int2*>(p.grid) + q);
-        sgrid[q] = grid_code<C::DF>(raw);
+        if (C::IQ2) reinterpret_cast<uint2*>(sgrid)[q] = grid_selectors(raw);
+        else sgrid[q] = grid_masks(raw);
         grid_bad |= !grid_row_ok<C::DF>(raw);
     }
     if (active) {
@@ -423,11 +448,6 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
         __syncthreads();  // panel g has landed; every thread is done with the other buffer
         prefetch(g + 1);
         const float* Hp = panel(g);
-        // this thread's 16-byte chunks of the panel it staged must be finite
-        for (int i = tid; i < W * kBlock / 4; i += kThreads) {
-            const float4 v = reinterpret_cast<const float4*>(Hp)[i];
-            h_bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
-        }
         if (active) {
             float dl[W];
             delta_of(g, dl);
@@ -461,6 +481,24 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     for (int rr = 0; rr < 4; ++rr)
         *reinterpret_cast<float4*>(grad_row(4 * rg + rr) + 4 * cg) =
             make_float4(gacc[rr][0].x, gacc[rr][0].y, gacc[rr][1].x, gacc[rr][1].y);
+    // Every entry H[k][i] of the block enters column i's gradient chain of every row (inactive
+    // rows with Delta = 0), and a non-finite product (inf * 0 is NaN) keeps the chain non-finite,
+    // so a finite gradient tile everywhere proves the block finite. A non-finite one (which a
+    // non-finite Delta or an overflow can also cause) sends the CTA to the exact scan of H.
+    {
+        bool tile_bad = false;
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+            tile_bad |= !(isfinite(gacc[rr][0].x) && isfinite(gacc[rr][0].y) && isfinite(gacc[rr][1].x) &&
+                          isfinite(gacc[rr][1].y));
+        if (__syncthreads_or(tile_bad)) {
+            const float4* H4 = reinterpret_cast<const float4*>(H);
+            for (int i = tid; i < kBlock * kBlock / 4; i += kThreads) {
+                const float4 v = __ldg(H4 + i);
+                h_bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+            }
+        }
+    }
     grid_bad = __syncthreads_or(grid_bad);
     h_bad = __syncthreads_or(h_bad);
     if (tid == 0) raise_flags(p.flags, (grid_bad ? IQ_FLAG_GRID : 0u) | (h_bad ? IQ_FLAG_NONFINITE : 0u));
@@ -496,7 +534,6 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
         if (active) {
             float dl[W], u[W];
             delta_of(g, dl);
-#pragma unroll
             {
                 float cg[W];
                 load_vec<W>(cur_row + g * W, cg);
