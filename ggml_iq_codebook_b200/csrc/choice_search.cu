@@ -236,16 +236,16 @@ __device__ __forceinline__ void half_argmin(float v, int /*c*/, unsigned mask, f
 }
 
 // v[i] = sum over k < W (fma chain, k ascending, starting from the product) of
-// Hp[k][col0 + i] * a[k], for NO columns. Adjacent columns run as one packed fma.rn.f32x2 (two
-// independent IEEE fmas, so every chain rounds exactly as the scalar one); the next panel row is
-// loaded while the current one is used.
-template <int W, int NO>
+// Hp[k][col0 + i] * a[k], for NO columns, Hp's rows LD floats apart. Adjacent columns run as one
+// packed fma.rn.f32x2 (two independent IEEE fmas, so every chain rounds exactly as the scalar
+// one); the next row is loaded while the current one is used.
+template <int W, int NO, int LD>
 __device__ __forceinline__ void group_matvec(const float* Hp, int col0, const float a[W], float v[NO]) {
     static_assert(NO % 4 == 0, "16-byte panel reads");
     float h[NO], hn[NO];
     float2 acc[NO / 2];
     load_vec<NO>(Hp + col0, h);
-    load_vec<NO>(Hp + kBlock + col0, hn);
+    load_vec<NO>(Hp + LD + col0, hn);
     {
         const float2 a0 = make_float2(a[0], a[0]);
 #pragma unroll
@@ -255,7 +255,7 @@ __device__ __forceinline__ void group_matvec(const float* Hp, int col0, const fl
     for (int k = 1; k < W; ++k) {
 #pragma unroll
         for (int i = 0; i < NO; ++i) h[i] = hn[i];
-        if (k + 1 < W) load_vec<NO>(Hp + (k + 1) * kBlock + col0, hn);
+        if (k + 1 < W) load_vec<NO>(Hp + (k + 1) * LD + col0, hn);
         const float2 ak = make_float2(a[k], a[k]);
 #pragma unroll
         for (int t = 0; t < NO / 2; ++t) acc[t] = __ffma2_rn(make_float2(h[2 * t], h[2 * t + 1]), ak, acc[t]);
@@ -300,10 +300,12 @@ __device__ __forceinline__ float join_parts(float t, unsigned mask) {
 
 // u^T H_gg u over this lane's candidate: (H_gg u) for this lane's columns, the products with u,
 // and the pairwise tree over the group's W columns (joined across the lanes of a candidate).
-template <int W, int WO, int SPLIT, int NC>
-__device__ __forceinline__ float quad_form(const float* Hp, int g, int part, const float u[W], unsigned mask) {
+// Hg is H_gg's first row, the group's first column at col0, rows LD floats apart: a panel
+// (LD = 256, col0 = g W) or a staged diagonal block (LD = W, col0 = 0).
+template <int W, int WO, int SPLIT, int NC, int LD>
+__device__ __forceinline__ float quad_form(const float* Hg, int col0, int part, const float u[W], unsigned mask) {
     float v[WO], up[WO];
-    group_matvec<W, WO>(Hp, g * W + part * WO, u, v);
+    group_matvec<W, WO, LD>(Hg, col0 + part * WO, u, v);
     lane_part<W, WO>(u, part, up);
 #pragma unroll
     for (int i = 0; i < WO; ++i) v[i] = __fmul_rn(up[i], v[i]);
@@ -439,19 +441,25 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
         return reinterpret_cast<float*>(smem + C::oRows + r * C::rBytes + C::rGrad);
     };
 
-    // ---- step 2 (each group's own diagonal block), fused with the initial gradient grad = H Delta
-    // and with the first sweep's curvature terms: u = Delta(c) - Delta(pick) changes only when
-    // group g itself switches, so u^T H_gg u is scored here, once, while panel g is resident.
-    float2 gacc[4][2];
-    for (int g = 0; g < G; ++g) {
-        cp_async_wait_all();
-        __syncthreads();  // panel g has landed; every thread is done with the other buffer
-        prefetch(g + 1);
-        const float* Hp = panel(g);
-        if (active) {
+    // ---- step 2: each group's pick from its own diagonal block, and the first sweep's curvature
+    // terms (u = Delta(c) - Delta(pick) changes only when group g itself switches, so u^T H_gg u is
+    // scored here, once). The G diagonal blocks H_gg (G W^2 floats, one panel buffer) are staged
+    // together in buffer 1 while panel 0 streams into buffer 0, so each row runs its G groups
+    // without waiting for the other rows.
+    float* Hd = panel(1);
+    for (int i = tid; i < G * W * W / 4; i += kThreads) {
+        const int gk = i / (W / 4), c4 = i % (W / 4);  // H row gk = g W + k, its 16-byte chunk c4 of H_gg
+        cp_async16(Hd + gk * W + 4 * c4, H + gk * kBlock + (gk / W) * W + 4 * c4);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    if (active) {
+        for (int g = 0; g < G; ++g) {
+            const float* Hg = Hd + g * W * W;
             float dl[W];
             delta_of(g, dl);
-            const float sq = quad_form<W, WO, C::SPLIT, NC>(Hp, g, part, dl, hmask);  // every lane joins
+            const float sq = quad_form<W, WO, C::SPLIT, NC, W>(Hg, 0, part, dl, hmask);  // every lane joins
             const float score = c < NC ? sq : INFINITY;
             float best;
             int cstar;
@@ -464,12 +472,20 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
             // the winner's Delta by shuffles, then u = Delta(c) - Delta(pick) in place
 #pragma unroll
             for (int i = 0; i < W; ++i) dl[i] = __fsub_rn(dl[i], __shfl_sync(hmask, dl[i], cstar, 16));
-            const float t2 = quad_form<W, WO, C::SPLIT, NC>(Hp, g, part, dl, hmask);
+            const float t2 = quad_form<W, WO, C::SPLIT, NC, W>(Hg, 0, part, dl, hmask);
             if (part == 0) t2row[g * NC + ch] = t2;
         }
-        __syncthreads();
-        // grad_i += H[k][i] cur_k over this group's k: a 4-row x 4-column tile per thread, fed by
-        // one 16-byte read of the rows' cur_k and one of H[k][4 columns] per k
+    }
+
+    // ---- the initial gradient grad = H Delta(picks), panel by panel: grad_i += H[k][i] cur_k over
+    // group g's k, a 4-row x 4-column tile per thread, fed by one 16-byte read of the rows' cur_k
+    // and one of H[k][4 columns] per k
+    float2 gacc[4][2];
+    for (int g = 0; g < G; ++g) {
+        if (g > 0) cp_async_wait_all();
+        __syncthreads();  // panel g has landed; every thread is done with the other buffer (or Hd)
+        prefetch(g + 1);
+        const float* Hp = panel(g);
 #pragma unroll 4
         for (int k = 0; k < W; ++k) {
             const float4 cv = *reinterpret_cast<const float4*>(curT + (g * W + k) * kRows + 4 * rg);
@@ -569,7 +585,7 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
                 if (step < 2 * G) {  // the second sweep's curvature terms around the new pick
 #pragma unroll
                     for (int i = 0; i < W; ++i) dl[i] = __fsub_rn(dl[i], __shfl_sync(hmask, dl[i], cstar, 16));
-                    const float t2 = quad_form<W, WO, C::SPLIT, NC>(Hp, g, part, dl, hmask);
+                    const float t2 = quad_form<W, WO, C::SPLIT, NC, kBlock>(Hp, g * W, part, dl, hmask);
                     if (part == 0) t2row[g * NC + ch] = t2;
                 }
             }
