@@ -24,21 +24,20 @@
 // set r / rows_per_hess (PR #3218's reason for one launch: thousands of small expert weights).
 //
 // Design (B200): one CTA = 16 rows (8 for IQ1_S) of one block, a half-warp per row and one lane per
-// choice. The rows run the group steps in lockstep, so each step stages one panel of H (the group's
-// W rows, W x 256 fp32) in shared memory once for all rows, double-buffered with cp.async so the
-// next panel streams in while this one is used; H is read from L2 three times per CTA (step 2 fused
-// with the initial gradient, then one pass per sweep). A lane decodes its own candidate's group
-// straight into registers and keeps all W accumulators of H_gg u: W independent fma chains fed by
-// broadcast 16-byte panel reads. Its two trees are local, and the only cross-lane step is a 4-level
-// argmin over the half-warp; the winning lane writes cur and u from its registers. The gradient
-// work (the initial H Delta, and after every sweep step the updates of the rows that switched) is
-// done by all threads together: the initial H Delta as 4-row x 4-column register tiles (per k one
-// 16-byte read of the rows' values and one of H, then 16 fmas); after a sweep step, by column when
-// few rows switched (each thread holding its H column and walking only those rows), else by the
-// same tiles. The grid is staged per format so that decoding needs no int-to-float conversion:
-// IQ1 as 16-bit +1/-1 masks, each element selecting among its group's three values; IQ2 as
-// byte-permute selectors over tables of the four magnitudes' 16-bit halves (two permutes per
-// pair of halves, two to join them into floats, the signs by XOR). The block's H is checked for
+// choice. Step 2 first stages all G diagonal blocks H_gg together (they fill one panel buffer), so
+// each row scores its groups with no CTA barrier: a lane decodes its own candidate's group straight
+// into registers and keeps all W accumulators of H_gg u, W independent fma chains fed by broadcast
+// 16-byte reads; its two trees are local, and the only cross-lane step is the argmin over the
+// half-warp. The initial gradient H Delta then streams H panel by panel (the group's W rows, W x 256
+// fp32, double-buffered with cp.async) as 4-row x 4-column register tiles (per k one 16-byte read
+// of the rows' values and one of H, then 16 fmas). The sweeps run the rows in lockstep over the same
+// panel stream, so each panel is staged once for all rows: each row decides from its stored
+// curvature terms and its gradient, and the gradients of the rows that switched are updated by all
+// threads, a column pair per thread in packed fmas. H is read from L2 three times per CTA, plus
+// its diagonal blocks once. The grid is staged per format so that decoding needs no int-to-float
+// conversion: IQ1 as 16-bit +1/-1 masks, each element selecting among its group's three values;
+// IQ2 as byte-permute selectors over tables of the four magnitudes' 16-bit halves (two permutes
+// per pair of halves, two to join them into floats, the signs by XOR). The block's H is checked for
 // non-finite entries through the initial gradient: every entry enters a chain of every row, so
 // the explicit scan runs only in a CTA whose gradient came out non-finite. On request each row's
 // final Delta^T H Delta is reported as sum_i cur_i grad_i (a pairwise tree over the 256 columns).
@@ -170,9 +169,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 
-constexpr int kColumnMaxW16 = 12;  // 16- and 8-column choice groups, 16 rows per CTA
-constexpr int kColumnMaxW32 = 0;   // 32-column choice groups (IQ1_S): always tiles (measured)
-
 template <int FMT>
 struct Cfg {
     static constexpr bool G8 = FMT == kChoiceIq2xsG8;          // eight candidates per 8-weight group
@@ -195,12 +191,9 @@ struct Cfg {
     // shared memory layout (bytes)
     static constexpr int oHp = 0;                             // float [2][W][256], double buffer
     static constexpr int oCurT = oHp + 2 * W * kBlock * 4;    // float [256][R]: the rows' current Delta
-    static constexpr int oUT = oCurT + kBlock * R * 4;        // float [W][R]: u of the rows that switched
-    static constexpr int oUR = oUT + W * R * 4;               // float [R][W]: the same, by row
+    static constexpr int oUR = oCurT + kBlock * R * 4;        // float [R][W]: u of the rows that switched
     static constexpr int oT2 = oUR + R * W * 4;               // float [R][G][NC]: u^T H_gg u per candidate
     static constexpr int oSw = oT2 + R * G * NC * 4;          // uint32 [2]: rows that switched, by step parity
-    // update by column up to this many switched rows, else by tiles (either is bit-exact)
-    static constexpr int COLUMN_MAX = W == 32 ? kColumnMaxW32 : kColumnMaxW16;
     static constexpr bool IQ2 = DF == IQ_FMT_IQ2_XS || DF == IQ_FMT_IQ2_S;
     static constexpr int oGrid = oSw + R * 4;  // IQ2: uint2 [E] selectors; IQ1: uint16 [E] masks
     static constexpr int oRows = oGrid + (IQ2 ? E * 8 : (E * 2 + 15) / 16 * 16);  // per-row records
@@ -344,7 +337,6 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     static_assert(kThreads == C::RG * 64, "gradient tiles: 4 rows x 4 columns per thread");
     extern __shared__ __align__(16) char smem[];
     float* curT = reinterpret_cast<float*>(smem + C::oCurT);
-    float* uT = reinterpret_cast<float*>(smem + C::oUT);
     float* uR = reinterpret_cast<float*>(smem + C::oUR);
     uint32_t* swbits = reinterpret_cast<uint32_t*>(smem + C::oSw);
     uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem + C::oGrid);
@@ -573,8 +565,6 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
             if (switched) {
                 if (c == cstar) {
 #pragma unroll
-                    for (int i = 0; i < W; ++i) uT[i * kRows + hr] = u[i];
-#pragma unroll
                     for (int i = 0; i < W; i += 4)
                         *reinterpret_cast<float4*>(uR + hr * W + i) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
 #pragma unroll
@@ -592,48 +582,31 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
         }
         if (c == 0 && switched) atomicOr(&swbits[step & 1], 1u << hr);
         __syncthreads();
-        // grad[r][i] += sum_k H[k][i] u_k (fma chain over the group's k, the same order either
-        // way) for the rows that switched. Few switches: by column, each thread holding H[k][i]
-        // for its columns in registers and walking only those rows. Many: 4-row x 4-column
-        // register tiles over every 4-row group with a switch, writing back only switched rows.
+        // grad[r][i] += sum_k H[k][i] u_k (fma chain over the group's k) for the rows that
+        // switched: a column pair per thread, its H[k][2 cp .. 2 cp + 1] in registers, as two
+        // independent chains in packed fmas; the CTA's thread sets split the switched rows by
+        // their rank among them. (Register tiles over 4-row groups measured no faster for IQ2 and
+        // 5% slower for IQ1_S.)
         const uint32_t swmask = swbits[step & 1];
         if (tid == 0) swbits[(step + 1) & 1] = 0u;  // every thread read it last step, before this step's first barrier
-        if (swmask != 0 && __popc(swmask) <= C::COLUMN_MAX) {
+        if (swmask != 0) {
+            constexpr int kSets = kThreads / (kBlock / 2);
+            const int cp = tid % (kBlock / 2), set = tid / (kBlock / 2);
+            float2 hcol[W];
 #pragma unroll
-            for (int i = tid; i < kBlock; i += kThreads) {
-                float hcol[W];
+            for (int k = 0; k < W; ++k) hcol[k] = *reinterpret_cast<const float2*>(Hp + k * kBlock + 2 * cp);
+            int rank = 0;
+            for (uint32_t m = swmask; m != 0; m &= m - 1, ++rank) {
+                if (rank % kSets != set) continue;
+                const int r = __ffs(m) - 1;
+                float uk[W];
+                load_vec<W>(uR + r * W, uk);
+                float2* gr = reinterpret_cast<float2*>(grad_row(r)) + cp;
+                float2 acc = *gr;
 #pragma unroll
-                for (int k = 0; k < W; ++k) hcol[k] = Hp[k * kBlock + i];
-                for (uint32_t m = swmask; m != 0; m &= m - 1) {
-                    const int r = __ffs(m) - 1;
-                    float uk[W];
-                    load_vec<W>(uR + r * W, uk);
-                    float* gr = grad_row(r);
-                    float acc = gr[i];
-#pragma unroll
-                    for (int k = 0; k < W; ++k) acc = __fmaf_rn(hcol[k], uk[k], acc);
-                    gr[i] = acc;
-                }
+                for (int k = 0; k < W; ++k) acc = __ffma2_rn(hcol[k], make_float2(uk[k], uk[k]), acc);
+                *gr = acc;
             }
-        } else if (swmask != 0 && ((swmask >> (4 * rg)) & 15u) != 0) {
-            float2 acc[4][2];
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                const float4 a = *reinterpret_cast<const float4*>(grad_row(4 * rg + rr) + 4 * cg);
-                acc[rr][0] = make_float2(a.x, a.y);
-                acc[rr][1] = make_float2(a.z, a.w);
-            }
-#pragma unroll 4
-            for (int k = 0; k < W; ++k) {
-                const float4 uv = *reinterpret_cast<const float4*>(uT + k * kRows + 4 * rg);
-                const float4 hv = *reinterpret_cast<const float4*>(Hp + k * kBlock + 4 * cg);
-                tile_fma(acc, hv, uv, false);
-            }
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr)
-                if ((swmask >> (4 * rg + rr)) & 1u)  // rows that kept their choice keep their gradient
-                    *reinterpret_cast<float4*>(grad_row(4 * rg + rr) + 4 * cg) =
-                        make_float4(acc[rr][0].x, acc[rr][0].y, acc[rr][1].x, acc[rr][1].y);
         }
     }
 
