@@ -31,13 +31,13 @@ DEFAULT_ANCHOR = {"iq1_s": 0.61, "iq2_xs": 0.9, "iq1_m": 1.0, "iq2_s": 0.9}
 
 IQ_OUT_F32, IQ_OUT_BF16 = 0, 1
 IQ_IN = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
-FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID = 1, 2, 4, 8, 16
+FLAG_NONFINITE, FLAG_IMPORTANCE, FLAG_RANGE, FLAG_CHOICE, FLAG_GRID, FLAG_TIMEOUT = 1, 2, 4, 8, 16, 32
 
 SYMBOLS = ("iq_block_bytes", "iq_payload_bytes", "iq_choice_groups", "iq_num_choices", "iq_encode", "iq_decode",
            "iq_choice_search", "iq_choice_search_g8", "iq_gptq_workspace_bytes", "iq_gptq_blocks",
            "iq_gptq_blocks_static", "iq_sqrt_diag",
            "iq_status_string", "iq_build_info")
-PROBE_SYMBOLS = ("iq_probe_fp32", "iq_probe_fp32_ops_per_iter")  # include/iq_probe.h: measurement only
+PROBE_SYMBOLS = ("iq_probe_fp32", "iq_probe_fp32_ops_per_iter", "iq_probe_bulk_wait")  # include/iq_probe.h
 
 
 class IQError(RuntimeError):
@@ -95,6 +95,8 @@ def load_library(path: str = LIB_PATH):
     lib.iq_probe_fp32.argtypes = [i32, i64, i64, P, P]
     lib.iq_probe_fp32_ops_per_iter.restype = i64
     lib.iq_probe_fp32_ops_per_iter.argtypes = [i32]
+    lib.iq_probe_bulk_wait.restype = i32
+    lib.iq_probe_bulk_wait.argtypes = [P, i64, i32, i64, P, P]
     _lib = lib
     return lib
 
@@ -207,7 +209,8 @@ def raise_for_flags(flags: torch.Tensor) -> None:
     if f:
         names = [n for n, b in (("non-finite weight", FLAG_NONFINITE), ("bad importance", FLAG_IMPORTANCE),
                                 ("d overflows fp16", FLAG_RANGE), ("choice out of range", FLAG_CHOICE),
-                                ("grid value outside the alphabet", FLAG_GRID)) if f & b]
+                                ("grid value outside the alphabet", FLAG_GRID),
+                                ("a bounded copy wait ran out", FLAG_TIMEOUT)) if f & b]
         err = IQError("device-side finding: " + ", ".join(names))
         err.flags = f
         raise err
@@ -417,6 +420,17 @@ def probe_fp32(kind: str, blocks: int, iters: int, out: torch.Tensor, stream=Non
     if lib.iq_probe_fp32(k, blocks, iters, out.data_ptr(), _stream(stream)) != 0:
         raise IQError("iq_probe_fp32 failed")
     return blocks * 256 * iters * int(lib.iq_probe_fp32_ops_per_iter(k))
+
+
+def probe_bulk_wait(src: torch.Tensor | None, arm: bool, limit_cycles: int, out: torch.Tensor, stream=None) -> None:
+    """Launch the bulk-copy wait check (include/iq_probe.h): out[0] = 1 if the wait completed in
+    time, out[1] = the weighted word sum of what was copied."""
+    lib = load_library()
+    _need(out, torch.int32, "out")
+    nbytes = 0 if src is None else src.numel() * src.element_size()
+    if lib.iq_probe_bulk_wait(None if src is None else src.data_ptr(), nbytes, int(arm), limit_cycles,
+                              out.data_ptr(), _stream(stream)) != 0:
+        raise IQError("iq_probe_bulk_wait failed")
 
 
 def build_info() -> str:

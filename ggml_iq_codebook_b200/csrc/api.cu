@@ -90,13 +90,15 @@ class FlagsWord {
     uint32_t* ptr() const { return caller_ != nullptr ? caller_ : own_; }
     // The call's status: `st` itself when the launch failed or the caller keeps the word;
     // otherwise the library's word is read once the stream is done, and a finding becomes
-    // IQ_EGRID, IQ_ENONFINITE, IQ_EIMPORTANCE, IQ_ERANGE or IQ_ECHOICE (first match wins).
+    // IQ_ETIMEOUT, IQ_EGRID, IQ_ENONFINITE, IQ_EIMPORTANCE, IQ_ERANGE or IQ_ECHOICE (first match
+    // wins).
     iq_status finish(iq_status st, cudaStream_t s) {
         if (st != IQ_OK || caller_ != nullptr) return st;
         uint32_t f = 0;
         if (cudaMemcpyAsync(&f, own_, sizeof(f), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
             cudaStreamSynchronize(s) != cudaSuccess)
             return IQ_ECUDA;
+        if (f & IQ_FLAG_TIMEOUT) return IQ_ETIMEOUT;
         if (f & IQ_FLAG_GRID) return IQ_EGRID;
         if (f & IQ_FLAG_NONFINITE) return IQ_ENONFINITE;
         if (f & IQ_FLAG_IMPORTANCE) return IQ_EIMPORTANCE;
@@ -411,6 +413,7 @@ const char* iq_status_string(iq_status s) {
         case IQ_ECHOICE: return "a given choice is out of the format's range";
         case IQ_EGRID: return "a grid value lies outside the format's alphabet";
         case IQ_ESCRATCH: return "the call needs more scratch than the library's static 10 MiB array";
+        case IQ_ETIMEOUT: return "a kernel's bounded wait for its own copy ran out";
         default: return "unknown status";
     }
 }

@@ -29,8 +29,9 @@
 // into registers and keeps all W accumulators of H_gg u, W independent fma chains fed by broadcast
 // 16-byte reads; its two trees are local, and the only cross-lane step is the argmin over the
 // half-warp. The initial gradient H Delta then streams H panel by panel (the group's W rows, W x 256
-// fp32, double-buffered with cp.async) as 4-row x 4-column register tiles (per k one 16-byte read
-// of the rows' values and one of H, then 16 fmas). The sweeps run the rows in lockstep over the same
+// contiguous fp32, double-buffered; one thread issues each panel as one bulk copy that completes
+// on the buffer's mbarrier, every thread waits with a bound) as 4-row x 4-column register tiles
+// (per k one 16-byte read of the rows' values and one of H, then 16 fmas). The sweeps run the rows in lockstep over the same
 // panel stream, so each panel is staged once for all rows: each row decides from its stored
 // curvature terms and its gradient, and the gradients of the rows that switched are updated by all
 // threads, a column pair per thread in packed fmas. H is read from L2 three times per CTA, plus
@@ -195,7 +196,8 @@ struct Cfg {
     static constexpr int oT2 = oUR + R * W * 4;               // float [R][G][NC]: u^T H_gg u per candidate
     static constexpr int oSw = oT2 + R * G * NC * 4;          // uint32 [2]: rows that switched, by step parity
     static constexpr bool IQ2 = DF == IQ_FMT_IQ2_XS || DF == IQ_FMT_IQ2_S;
-    static constexpr int oGrid = oSw + R * 4;  // IQ2: uint2 [E] selectors; IQ1: uint16 [E] masks
+    static constexpr int oBar = oSw + R * 4;   // uint64 [2] panel barriers, uint32 abort word
+    static constexpr int oGrid = oBar + 32;    // IQ2: uint2 [E] selectors; IQ1: uint16 [E] masks
     static constexpr int oRows = oGrid + (IQ2 ? E * 8 : (E * 2 + 15) / 16 * 16);  // per-row records
     static constexpr int rGrad = 0;                               // float [256]
     static constexpr int rPick = rGrad + kBlock * 4;              // int [G]
@@ -339,6 +341,8 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     float* curT = reinterpret_cast<float*>(smem + C::oCurT);
     float* uR = reinterpret_cast<float*>(smem + C::oUR);
     uint32_t* swbits = reinterpret_cast<uint32_t*>(smem + C::oSw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::oBar);
+    volatile uint32_t* abort_word = reinterpret_cast<volatile uint32_t*>(smem + C::oBar + 16);
     uint16_t* sgrid = reinterpret_cast<uint16_t*>(smem + C::oGrid);
 
     // CTA -> (block, expert, row tile): a tile never straddles two experts, and the CTAs that
@@ -364,16 +368,29 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     const void* xrow = F32 ? static_cast<const void*>(static_cast<const float*>(p.w) + row * p.ldw + blk * kBlock)
                            : static_cast<const void*>(static_cast<const uint16_t*>(p.w) + row * p.ldw + blk * kBlock);
 
-    // H panels (the W rows of one choice group) stream through a double buffer: step s of the
-    // 3G group steps (step 2, then two sweeps) uses panel s % G from buffer s & 1.
+    // H panels (the W rows of one choice group, W x 256 contiguous fp32) stream through a double
+    // buffer: step s of the 3G panel steps (the initial gradient, then two sweeps) uses panel
+    // s % G from buffer s & 1. One thread issues each panel as one bulk copy completing on the
+    // buffer's barrier; every thread waits for that phase (parity (s >> 1) & 1, the buffer's
+    // (s >> 1)-th use) with a bound. A wait that runs out marks the CTA aborted: its waits stop,
+    // and its row-blocks are written as findings (IQ_FLAG_TIMEOUT).
     auto panel = [&](int step) { return reinterpret_cast<float*>(smem + C::oHp + (step & 1) * W * kBlock * 4); };
-    auto prefetch = [&](int step) {
-        const char* src = reinterpret_cast<const char*>(H + (step % G) * W * kBlock);
-        char* dst = reinterpret_cast<char*>(panel(step));
-        for (int i = tid; i < W * kBlock / 4; i += kThreads) cp_async16(dst + 16 * i, src + 16 * i);
-        cp_async_commit();
+    auto prefetch = [&](int step) {  // thread 0, after a CTA barrier that freed the buffer
+        bulk_load(panel(step), H + (step % G) * W * kBlock, W * kBlock * 4, bars + (step & 1));
     };
-    prefetch(0);
+    bool timed_out = false;
+    auto wait_panel = [&](int step) {
+        if (*abort_word == 0u && !mbar_wait(bars + (step & 1), (step >> 1) & 1, kBulkWaitCycles)) {
+            timed_out = true;
+            *abort_word = 1u;
+        }
+    };
+    if (tid == 0) {
+        mbar_init(bars);
+        mbar_init(bars + 1);
+        *abort_word = 0u;
+        prefetch(0);
+    }
 
     // ---- stage the grid (checking the alphabet) and the row's candidate payloads (lanes
     // past the format's NC candidates stage zeros and never win); a non-finite weight taints the row
@@ -474,9 +491,9 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     // and one of H[k][4 columns] per k
     float2 gacc[4][2];
     for (int g = 0; g < G; ++g) {
-        if (g > 0) cp_async_wait_all();
-        __syncthreads();  // panel g has landed; every thread is done with the other buffer (or Hd)
-        prefetch(g + 1);
+        __syncthreads();  // every thread is done with the other buffer (panel g - 1, or Hd)
+        if (tid == 0) prefetch(g + 1);
+        wait_panel(g);
         const float* Hp = panel(g);
 #pragma unroll 4
         for (int k = 0; k < W; ++k) {
@@ -534,9 +551,9 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
     // updates its gradient tile for the rows that switched.
     for (int step = G; step < 3 * G; ++step) {
         const int g = step % G;
-        cp_async_wait_all();
         __syncthreads();
-        if (step + 1 < 3 * G) prefetch(step + 1);
+        if (tid == 0 && step + 1 < 3 * G) prefetch(step + 1);
+        wait_panel(step);
         const float* Hp = panel(step);
         int switched = 0;
         if (active) {
@@ -610,11 +627,18 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
         }
     }
 
-    __syncthreads();  // every gradient update has landed
+    // every gradient update has landed; an aborted CTA waits once more (bounded) for copies in flight
+    const bool cta_timed_out = __syncthreads_or(timed_out);
+    if (cta_timed_out && tid == 0) {
+        const int last = 3 * G - 1;  // the last panel step; its barrier phase and the other buffer's
+        mbar_wait(bars + (last & 1), (last >> 1) & 1, kBulkWaitCycles);
+        mbar_wait(bars + ((last - 1) & 1), ((last - 1) >> 1) & 1, kBulkWaitCycles);
+        raise_flags(p.flags, IQ_FLAG_TIMEOUT);
+    }
     // A row-block with a finding (a non-finite weight in the row, a non-finite entry in its
-    // Hessian block, a grid value outside the alphabet) reports picks 0, the all-zero payload and
-    // a NaN objective.
-    const bool tainted = grid_bad || h_bad || row_bad;
+    // Hessian block, a grid value outside the alphabet, a copy wait that ran out) reports picks 0,
+    // the all-zero payload and a NaN objective.
+    const bool tainted = grid_bad || h_bad || row_bad || cta_timed_out;
 
     // ---- the final objective Delta^T H Delta = sum_i cur_i grad_i: lane c sums columns
     // 16c .. 16c + 15 by a pairwise tree, then the butterfly joins the 16 lanes pairwise

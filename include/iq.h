@@ -39,8 +39,8 @@
  *     the word holds exactly this call's findings; the status only covers the host-side checks.
  *   - flags == NULL: the call is SYNCHRONOUS. The kernels report into a word the library keeps on
  *     each device; the call waits for `stream` to finish it and returns the first finding as a
- *     status (IQ_EGRID, IQ_ENONFINITE, IQ_EIMPORTANCE, IQ_ERANGE, IQ_ECHOICE, in that order of
- *     precedence), so bad data never comes back as IQ_OK. Such calls on one device are serialised
+ *     status (IQ_ETIMEOUT, IQ_EGRID, IQ_ENONFINITE, IQ_EIMPORTANCE, IQ_ERANGE, IQ_ECHOICE, in that
+ *     order of precedence), so bad data never comes back as IQ_OK. Such calls on one device are serialised
  *     by a host mutex held from clearing that word to reading it back.
  *
  * Requires an sm_100 (B200-class) device; other devices get IQ_EUNSUPPORTED.
@@ -69,7 +69,8 @@ typedef enum {
     IQ_ERANGE = 7,        /* d rounds to fp16 infinity, or a given d is negative, infinite or NaN */
     IQ_ECHOICE = 8,       /* a given choice is >= the format's number of choices              */
     IQ_EGRID = 9,         /* a grid value lies outside the format's alphabet                   */
-    IQ_ESCRATCH = 10      /* iq_gptq_blocks_static: the call needs more than the library's 10 MiB */
+    IQ_ESCRATCH = 10,     /* iq_gptq_blocks_static: the call needs more than the library's 10 MiB */
+    IQ_ETIMEOUT = 11      /* a kernel's bounded wait for its own copy ran out (see IQ_FLAG_TIMEOUT) */
 } iq_status;
 
 typedef enum { IQ_FMT_IQ1_S = 1, IQ_FMT_IQ2_XS = 2, IQ_FMT_IQ1_M = 3, IQ_FMT_IQ2_S = 4 } iq_format;
@@ -86,6 +87,10 @@ typedef enum { IQ_IN_BF16 = 0, IQ_IN_F16 = 1, IQ_IN_F32 = 2 } iq_in_dtype;
 #define IQ_FLAG_RANGE 4u      /* d rounds to fp16 infinity, or a given d is < 0, inf or NaN */
 #define IQ_FLAG_CHOICE 8u     /* a given choice is >= 16                                  */
 #define IQ_FLAG_GRID 16u      /* a grid value lies outside the format's alphabet           */
+/* a CTA's bounded wait for one of its own bulk copies into shared memory ran out (about 0.1 s;
+ * not expected on a working device): its row-blocks are written as the all-zero payload with
+ * picks 0 and a NaN objective, and the CTA stops waiting */
+#define IQ_FLAG_TIMEOUT 32u
 
 /*
  * Codebook/convention descriptor (host struct; the grid it points to lives on the device).

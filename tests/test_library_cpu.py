@@ -53,9 +53,9 @@ def test_format_tables(lib):
         assert lib.iq_num_choices(code) == iq.CHOICES[fmt]
     assert b"sm_100a" in lib.iq_build_info()
     assert lib.iq_status_string(2).startswith(b"invalid shape")
-    for st in range(11):
+    for st in range(12):
         assert lib.iq_status_string(st) != b"unknown status", st
-    assert lib.iq_status_string(11) == b"unknown status"
+    assert lib.iq_status_string(12) == b"unknown status"
     assert lib.iq_probe_fp32_ops_per_iter(0) == 8 and lib.iq_probe_fp32_ops_per_iter(3) == 16
     assert lib.iq_probe_fp32_ops_per_iter(4) == 0
 
