@@ -547,8 +547,8 @@ __global__ void __launch_bounds__(Cfg<FMT>::T, 2) choice_search_kernel(const Cho
 
     // ---- step 3: two sweeps over the groups. Each row decides (lane per choice) from the stored
     // curvature term and the current gradient; a row that switches in the first sweep rescores
-    // that group's curvature terms around its new pick for the second. Then every thread
-    // updates its gradient tile for the rows that switched.
+    // that group's curvature terms around its new pick for the second. Then all threads update
+    // the switched rows' gradients, a column pair per thread.
     for (int step = G; step < 3 * G; ++step) {
         const int g = step % G;
         __syncthreads();
