@@ -67,9 +67,9 @@ def test_encode_without_flags_word_returns_the_finding(dev, grids, anchors):
     assert lib.iq_status_string(st).startswith(b"a grid value")
 
 
-def _choice_inputs(fmt, grids, anchors, dev, rows=20, nblk=2, seed=911):
+def _choice_inputs(fmt, grids, anchors, dev, rows=20, nblk=2, seed=911, std=0.02):
     base = "iq2_xs" if fmt == "g8" else fmt
-    w = synth.normal_bf16((rows, 256 * nblk), 0.02, seed)
+    w = synth.normal_bf16((rows, 256 * nblk), std, seed)
     hess = torch.stack([synth.block_hessian(seed + 10 + b, offdiag_std=0.3) for b in range(nblk)])
     imp = oracle.sqrt_diag(hess.numpy())
     cand, _ = oracle.encode(base, grids[base], anchors[base], w, importance=imp, every_choice=True)
@@ -144,3 +144,27 @@ def test_choice_search_refuses_ragged_width(dev, grids, anchors):
     cand = torch.zeros((16, 4, 1, 74), dtype=torch.uint8, device=dev)
     with pytest.raises(iq.IQError, match="multiple of 256"):
         iq.iq_choice_search(desc, w, hess, cand)
+
+
+@pytest.mark.parametrize("fmt", ["iq2_xs", "iq1_s"])
+def test_choice_search_overflowing_gradient_is_not_a_finding(dev, grids, anchors, fmt):
+    """A finite H whose products overflow fp32: the kernel's finiteness proof through the initial
+    gradient fails, its exact scan of H finds every entry finite, so nothing is flagged, and picks,
+    payload and objective still equal the oracle's (objective NaNs compared as NaN: their bit
+    patterns are the hardware's)."""
+    # unit-scale weights, so that H x Delta overflows once H sits near the top of the range
+    base, w, hess, cand = _choice_inputs(fmt, grids, anchors, dev, rows=12, nblk=2, seed=933, std=1.0)
+    desc = iq.make_desc(base, torch.from_numpy(grids[base]).to(dev), anchors[base])
+    big = hess.clone()
+    big[1] = big[1] * (3.0e38 / float(big[1].abs().max()))   # block 1 at the top of the fp32 range
+    assert torch.isfinite(big).all()
+    got = _gpu_search(fmt, base, desc, w, big, cand, dev)
+    want = _oracle_search(fmt, base, grids[base], w, big, cand)
+    assert got[3] == want[3] == 0
+    assert np.array_equal(got[0], want[0])
+    assert np.array_equal(got[1], want[1])
+    g_obj, w_obj = got[2], want[2]
+    assert np.array_equal(np.isnan(g_obj), np.isnan(w_obj))
+    ok = ~np.isnan(w_obj)
+    assert np.array_equal(g_obj[ok].view(np.uint32), w_obj[ok].view(np.uint32))
+    assert not np.isfinite(w_obj[:, 1]).all() and np.isfinite(w_obj[:, 0]).all()  # block 1 overflows
