@@ -235,6 +235,10 @@ WORKLOADS = {
                               "weighted payload x16)"),
     "iq2s_decode_1m_blocks": ("iq2_s", [8192, 4096], "IQ2_S bf16 decode of 1,048,576 blocks (the 8192x4096 "
                               "payload x8)"),
+    "iq1s_decode_4m_blocks": ("iq1_s", [4096, 4096], "IQ1_S bf16 decode of 4,194,304 blocks (the 4096x4096 "
+                              "weighted payload x64): a launch whose writes dwarf the L2"),
+    "iq2xs_decode_4m_blocks": ("iq2_xs", [8192, 4096], "IQ2_XS bf16 decode of 4,194,304 blocks (the 8192x4096 "
+                               "payload x32): a launch whose writes dwarf the L2"),
     "gptq_iq2xs_4096x4096": ("iq2_xs", [4096, 4096], "per-block calibration loop in one call: for each 256-column "
                              "block in order, sqrt(diag H_b) + IQ2_XS every-choice encode + two-sweep local-Hessian "
                              "search + GPTQ propagation of its error to the later columns; 4096x4096 bf16 "
@@ -281,14 +285,15 @@ class Workload:
                 self.launches_per_step = 2 + self.w.shape[-1] // 256
         elif name.startswith("gptq_"):
             self._gptq(synth.workload_gptq_iq2xs(), text)
-        elif name.endswith("_decode_1m_blocks"):
+        elif name.endswith("m_blocks") and "_decode_" in name:
             base = {"iq1s": synth.workload_iq1s_4096x4096_weighted(), "iq1m": dict(
                 synth.workload_iq1s_4096x4096_weighted(), fmt="iq1_m"), "iq2xs": synth.workload_iq2xs_8192x4096(),
                 "iq2s": dict(synth.workload_iq2xs_8192x4096(), fmt="iq2_s")}
             self._encode_decode(base[name.split("_")[0]], text)
             self.kind = "decode"
             B = iq.BLOCK_BYTES[self.fmt]
-            self.payload = self.payload.reshape(-1, B).repeat((1 << 20) // (self.payload.numel() // B), 1)
+            mblocks = int(name.split("_")[-2][:-1])  # 1 or 4 (x 2^20 blocks)
+            self.payload = self.payload.reshape(-1, B).repeat((mblocks << 20) // (self.payload.numel() // B), 1)
             self.decoded = torch.empty((self.payload.shape[0], 256), dtype=torch.bfloat16, device=self.dev)
             self.units = self.payload.shape[0] * 256
             self.nblocks = self.payload.shape[0]
@@ -510,12 +515,18 @@ def decode_roofline(wl: Workload, dev, peaks):
     nbytes = nblocks * (B + 512)
     gbs = nbytes / ms / 1e6
     del big, out, flush
-    name = {"iq1_s": "iq1s_decode_1m_blocks", "iq2_xs": "iq2xs_decode_1m_blocks", "iq1_m": "iq1m_decode_1m_blocks",
-            "iq2_s": "iq2s_decode_1m_blocks"}
-    if wl.fmt in name:
-        traffic, note = kernel_traffic("decode_kernel", name[wl.fmt], nblocks)
-    else:
-        traffic, note = None, f"no capture of the {wl.fmt} decode"
+    # the DRAM counters of a 4M-block launch where there is one (writes still in the L2 when a
+    # launch ends escape its counters, a smaller share of a larger launch), else of a 1M-block one
+    name = {"iq1_s": ["iq1s_decode_4m_blocks", "iq1s_decode_1m_blocks"],
+            "iq2_xs": ["iq2xs_decode_4m_blocks", "iq2xs_decode_1m_blocks"], "iq1_m": ["iq1m_decode_1m_blocks"],
+            "iq2_s": ["iq2s_decode_1m_blocks"]}
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    captured = set(json.load(open(tpath))) if os.path.exists(tpath) else set()
+    traffic, note = None, f"no capture of the {wl.fmt} decode"
+    for cand in name.get(wl.fmt, []):
+        if f"decode_kernel@{cand}" in captured:
+            traffic, note = kernel_traffic("decode_kernel", cand, nblocks)
+            break
     return {"kernel": "decode_kernel (bf16 out)", "blocks": nblocks, "bytes_per_launch": nbytes,
             "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
             "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic, "traffic_source": note}
@@ -566,6 +577,8 @@ def oracle_sample_rate(name: str, budget_s: float, rows_hint: int | None = None)
                   "iq1s_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
                   "iq1m_decode_1m_blocks": synth.workload_iq1s_4096x4096_weighted,
                   "iq2xs_decode_1m_blocks": synth.workload_iq2xs_8192x4096,
+                  "iq1s_decode_4m_blocks": synth.workload_iq1s_4096x4096_weighted,
+                  "iq2xs_decode_4m_blocks": synth.workload_iq2xs_8192x4096,
                   "iq2s_decode_1m_blocks": synth.workload_iq2xs_8192x4096,
                   "iq2xs_8192x4096": synth.workload_iq2xs_8192x4096,
                   "iq2s_8192x4096": synth.workload_iq2xs_8192x4096,
