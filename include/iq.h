@@ -223,7 +223,9 @@ iq_status iq_decode(const iq_desc *desc, const uint8_t *payload, int64_t nblocks
  * Findings (IQ_FLAG_NONFINITE: a non-finite weight in the row-block or a non-finite entry of its
  * Hessian block; IQ_FLAG_GRID: a grid value outside the candidates' alphabet) make that
  * row-block report picks 0 (the first candidate), the all-zero payload and a NaN objective
- * (bits 0x7FC00000); the other row-blocks are unaffected.
+ * (bits 0x7FC00000); the other row-blocks are unaffected. The kernel streams H in bulk copies
+ * and bounds every wait for them; a wait that runs out (IQ_FLAG_TIMEOUT, not expected on a
+ * working device) reports the row-blocks of its CTA the same way.
  */
 iq_status iq_choice_search(const iq_desc *desc, const uint16_t *w, int64_t rows, int64_t nblk,
                            int64_t ldw, const float *hess, int64_t rows_per_hess, const uint8_t *cand,
