@@ -39,8 +39,8 @@ METRIC = "IQ encode Mweights/s"
 UNIT = "Mweights/s"
 L2_FLUSH_BYTES = 256 << 20
 
-# FP32 operations the method itself requires, counted as the survey's work table counts them
-# (every candidate of the exhaustive search counts, an fma and a min one op each):
+# FP32 operations the method itself requires (the algorithmic work: every candidate of the
+# exhaustive search counts, an fma and a min one op each):
 #   IQ1_S, per 8-weight group: 2048 entries x 16 choices = 32,768 candidates x (fma + min) plus
 #     about 10 entry-term ops per entry (2048 x 10) = 86,016 ops; per 256-weight block x32 =
 #     2,752,512. IQ1_M runs the same search.
@@ -357,7 +357,7 @@ class Workload:
         self.text = text
         self.launches_per_step = 1 + 5 * nblk - 2  # fp32 copy; per block sqrt diag, encode, search, solve, update
         self.dominant = "per-block loop (every kernel of the call)"
-        # the survey's counts for the encode and the search, plus the propagation: the solve's
+        # the algorithmic counts for the encode and the search, plus the propagation: the solve's
         # 256 x 255 / 2 fmas per row-block and rows x 256 fmas per later column
         later = sum(cols - 256 * (b + 1) for b in range(nblk))
         self.ops_per_launch = (self.nblocks * (OPS_PER_BLOCK[self.fmt] + choice_ops_per_row_block(16) + 256 * 255 // 2)
@@ -743,8 +743,8 @@ def main():
         nominal = alu_peak_tops(peaks["sm_max_mhz"])
         roof = {"bound": "alu", "kernel": wl.dominant, "achieved": round(achieved, 3), "peak": peak,
                 "unit": "Top/s", "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_source": tnote,
-                "ops_per_launch": wl.ops_per_launch, "ops_count": "the survey's work table (every candidate "
-                "counts; fma and min one op each)", "ms_per_launch": round(dom_avg, 4),
+                "ops_per_launch": wl.ops_per_launch, "ops_count": "algorithmic work (every candidate of the "
+                "exhaustive search counts; fma and min one op each)", "ms_per_launch": round(dom_avg, 4),
                 "peak_basis": "measured in this run: FP32 lane ops/s of iq_probe_fp32 (8 CTAs x 256 threads per "
                 f"SM), the larger of scalar fma {fp32['ffma']} and packed fma.f32x2 {fp32['ffma2']} Top/s",
                 "peak_nominal": round(nominal, 3), "frac_of_nominal": round(achieved / nominal, 4)}
